@@ -1,0 +1,355 @@
+"""Pins of the CPU oracle against things other than itself: brute-force
+unrolling, closed forms, invariants, constructed selection cases, the pages'
+printed accounting, and directional quality claims.  CPU only."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import Cfg, Tile, exact_run, quantize, dequantize
+from recurrent_state_quantization_decode_b200 import workloads as wl
+
+
+def _inputs(rng, T, dk, dv, gate, unit_k=True, beta=None):
+    q = rng.standard_normal((T, dk))
+    k = rng.standard_normal((T, dk))
+    if unit_k:
+        k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((T, dv))
+    a = rng.uniform(0.8, 1.0, (T, dk if gate else 1))
+    b = rng.uniform(0.05, 1.0, T) if beta is None else np.full(T, float(beta))
+    return q, k, v, a, b
+
+
+def _relerr(x, ref):
+    return np.max(np.abs(x - ref)) / max(np.max(np.abs(ref)), 1e-300)
+
+
+# --------------------------------------------------------------------------
+# Exact recurrence
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("gate", [0, 1])
+@pytest.mark.parametrize("dk,dv", [(5, 3), (3, 6), (8, 8)])
+def test_exact_matches_product_form_unroll(gate, dk, dv):
+    """The oracle's delta-rule update against the product form
+    S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+    o_t = S_t q_t, written as explicit matrix products."""
+    rng = np.random.default_rng(1)
+    T = 4
+    S0 = rng.standard_normal((dv, dk))
+    q, k, v, a, b = _inputs(rng, T, dk, dv, gate, unit_k=False)
+    cfg = Cfg(dk, dv, gate=gate)
+    S_orc, o_orc = exact_run(cfg, S0, q, k, v, a, b)
+    S = S0.copy()
+    for t in range(T):
+        D = np.diag(a[t] if gate else np.full(dk, a[t, 0]))
+        P = np.eye(dk) - b[t] * np.outer(k[t], k[t])
+        S = S @ D @ P + b[t] * np.outer(v[t], k[t])
+        np.testing.assert_allclose(o_orc[t], S @ q[t], rtol=0, atol=1e-13 * np.abs(S).max())
+    np.testing.assert_allclose(S_orc, S, rtol=0, atol=1e-13 * np.abs(S).max())
+
+
+@pytest.mark.parametrize("gate", [0, 1])
+def test_exact_closed_forms(gate):
+    rng = np.random.default_rng(2)
+    dk, dv, T = 6, 4, 9
+    cfg = Cfg(dk, dv, gate=gate)
+    S0 = rng.standard_normal((dv, dk))
+    # beta = 0: pure decay, S_t = S0 diag(prod alpha)
+    q, k, v, a, b = _inputs(rng, T, dk, dv, gate, beta=0.0)
+    S, o = exact_run(cfg, S0, q, k, v, a, b)
+    G = np.ones(dk)
+    for t in range(T):
+        G = G * (a[t] if gate else a[t, 0])
+        np.testing.assert_allclose(o[t], (S0 * G) @ q[t], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(S, S0 * G, rtol=1e-13, atol=1e-14)
+    # beta = 1 and unit keys: the updated state maps k_t to v_t exactly
+    for t in range(T):
+        q1, k1, v1, a1, b1 = _inputs(rng, 1, dk, dv, gate, beta=1.0)
+        S, _ = exact_run(cfg, S, q1, k1, v1, a1, b1)
+        np.testing.assert_allclose(S @ k1[0], v1[0], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Windowed buffer algebra (identity quantization)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("gate", [0, 1])
+@pytest.mark.parametrize("W", [1, 3, 16])
+@pytest.mark.parametrize("K", [0, 4])
+@pytest.mark.parametrize("dk,dv", [(7, 5), (4, 9), (16, 16)])
+def test_identity_quantization_reproduces_exact(gate, W, K, dk, dv):
+    """With identity quantization (no rounding anywhere), any window length and
+    any number of compensator lines, the windowed decode equals the exact
+    recurrence: outputs, and the state after a final flush."""
+    rng = np.random.default_rng(3)
+    T = 41
+    S0 = rng.standard_normal((dv, dk)) * 0.3
+    q, k, v, a, b = _inputs(rng, T, dk, dv, gate)
+    cfg = Cfg(dk, dv, W=W, K=K, gate=gate, quant=0)
+    S_ex, o_ex = exact_run(cfg, S0, q, k, v, a, b)
+    tile = Tile(cfg, S0)
+    o = np.concatenate([tile.run(q[:13], k[:13], v[:13], a[:13], b[:13]),
+                        tile.run(q[13:], k[13:], v[13:], a[13:], b[13:])])
+    for t in range(T):
+        assert _relerr(o[t], o_ex[t]) < 1e-12
+    assert _relerr(tile.state(), S_ex) < 1e-12
+    tile.flush()
+    assert tile.n[0] == 0
+    assert _relerr(tile.base(), S_ex) < 1e-12
+    assert tile.diag[oracle.D_WY_RESIDUAL] < 1e-12
+    assert tile.diag[oracle.D_FOLDS] == T // W + (1 if T % W else 0)
+
+
+def test_wy_pair_matches_delta_in_int8_mode():
+    rng = np.random.default_rng(4)
+    dk = dv = 32
+    cfg = Cfg(dk, dv)
+    S0 = rng.standard_normal((dv, dk)) * 0.05
+    q, k, v, a, b = _inputs(rng, 80, dk, dv, 0)
+    tile = Tile(cfg, S0)
+    tile.run(q, k, v, a, b)
+    assert tile.diag[oracle.D_FOLDS] == 5
+    assert tile.diag[oracle.D_WY_RESIDUAL] < 1e-12
+
+
+@pytest.mark.parametrize("gate", [0, 1])
+def test_in_window_state_is_exact_with_quantization_on(gate):
+    """Quantization only happens at folds: inside a window, beta = 1 and unit
+    keys give S_t k_t = v_t exactly (to fp64 rounding)."""
+    rng = np.random.default_rng(5)
+    dk, dv = 12, 10
+    cfg = Cfg(dk, dv, W=16, gate=gate)
+    tile = Tile(cfg, rng.standard_normal((dv, dk)) * 0.1)
+    for t in range(15):
+        q, k, v, a, b = _inputs(rng, 1, dk, dv, gate, beta=1.0)
+        o = tile.run(q, k, v, a, b)
+        S = tile.state()
+        np.testing.assert_allclose(S @ k[0], v[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(o[0], S @ q[0], rtol=0, atol=1e-12)
+
+
+def test_kda_with_uniform_gate_equals_gdn():
+    rng = np.random.default_rng(6)
+    dk, dv, T = 16, 8, 40
+    S0 = rng.standard_normal((dv, dk)) * 0.1
+    q, k, v, a, b = _inputs(rng, T, dk, dv, 0)
+    g = Tile(Cfg(dk, dv, W=16, gate=0), S0)
+    kd = Tile(Cfg(dk, dv, W=16, gate=1), S0)
+    og = g.run(q, k, v, a, b)
+    ok = kd.run(q, k, v, np.repeat(a, dk, axis=1), b)
+    np.testing.assert_array_equal(og, ok)
+    np.testing.assert_array_equal(g.rec.Q, kd.rec.Q)
+
+
+# --------------------------------------------------------------------------
+# Quantizer
+# --------------------------------------------------------------------------
+
+def _noncomp_mask(cfg, cid):
+    mask = np.ones((cfg.dv, cfg.dk), dtype=bool)
+    for c in cid[:cfg.K]:
+        if c < cfg.dv:
+            mask[c, :] = False
+        else:
+            mask[:, c - cfg.dv] = False
+    return mask
+
+
+@pytest.mark.parametrize("smooth", [0.0, 0.5, 1.0])
+@pytest.mark.parametrize("dk,dv,K", [(32, 32, 4), (24, 40, 3), (128, 128, 4), (16, 16, 0)])
+def test_quantize_error_bound_and_codes(smooth, dk, dv, K):
+    rng = np.random.default_rng(7)
+    S = rng.standard_normal((dv, dk)) * np.exp(rng.standard_normal((1, dk)))  # uneven columns
+    S[3] *= 30.0
+    cfg = Cfg(dk, dv, K=K, smooth=smooth)
+    rec = quantize(cfg, S)
+    S32 = S.astype(np.float32).astype(np.float64)
+    recon = dequantize(cfg, rec)
+    mask = _noncomp_mask(cfg, rec.cid)
+    # compensator lines reproduce the fp32 state exactly
+    np.testing.assert_array_equal(recon[~mask], S32[~mask])
+    # every other entry is within half a step (plus fp32 rounding of the steps)
+    step = rec.sig.astype(np.float64)[:, None] * rec.m.astype(np.float64)[None, :]
+    err = np.abs(recon - S32)
+    assert np.all(err[mask] <= step[mask] * (0.5 + 1e-5) + np.abs(S32[mask]) * 1e-6)
+    assert rec.Q.min() >= -127 and rec.Q.max() <= 127
+    assert np.all(rec.Q[~mask] == 0)
+    live = np.abs(rec.Q).max(axis=1) > 0
+    assert np.all(np.abs(rec.Q[live]).max(axis=1) == 127)
+
+
+def test_quantize_column_and_row_scaling_invariance():
+    """Powers of two are exact in fp32, so: with full smoothing, scaling key
+    column j by 2^e_j scales m_j alone; without smoothing, scaling value row i
+    by 2^f_i scales sigma_i alone.  Codes stay identical.  Either would fail if
+    smoothing ran along rows or scales along columns."""
+    rng = np.random.default_rng(8)
+    dk, dv = 24, 16
+    S = rng.standard_normal((dv, dk))
+    e = rng.integers(-6, 7, dk).astype(np.float64)
+    f = rng.integers(-6, 7, dv).astype(np.float64)
+    c_full = Cfg(dk, dv, K=0, smooth=1.0)
+    r0, r1 = quantize(c_full, S), quantize(c_full, S * 2.0 ** e[None, :])
+    np.testing.assert_array_equal(r0.Q, r1.Q)
+    np.testing.assert_array_equal(r0.sig, r1.sig)
+    np.testing.assert_array_equal(r0.m.astype(np.float64) * 2.0 ** e, r1.m)
+    c_none = Cfg(dk, dv, K=0, smooth=0.0)
+    r0, r1 = quantize(c_none, S), quantize(c_none, S * 2.0 ** f[:, None])
+    np.testing.assert_array_equal(r0.Q, r1.Q)
+    np.testing.assert_array_equal(r0.m, np.ones(dk, np.float32))
+    np.testing.assert_array_equal(r0.sig.astype(np.float64) * 2.0 ** f, r1.sig)
+
+
+def test_smoothing_reduces_error_on_column_outliers():
+    rng = np.random.default_rng(9)
+    dk = dv = 64
+    S = rng.standard_normal((dv, dk)) * 0.01
+    S[:, :8] *= 50.0  # heavy key columns, more than the compensators take
+    errs = {}
+    for smooth in (0.0, 0.5):
+        cfg = Cfg(dk, dv, K=4, smooth=smooth)
+        errs[smooth] = np.linalg.norm(dequantize(cfg, quantize(cfg, S)) - S)
+    assert errs[0.5] < 0.7 * errs[0.0]
+
+
+def test_selection_greedy_with_recompute_and_ties():
+    """Constructed 3x3 case.  Energies: rows 100, 9, 16.25; columns 100, 4,
+    21.25.  Pick 1: row 0 ties column 0, rows first -> row 0.  Recompute:
+    column 0 drops to 0.  Pick 2: column 2 (21.25).  Recompute: row 2 = 4 ties
+    column 1 = 4 -> row 2.  Pick 4: nothing left, first untaken line -> row 1."""
+    S = np.array([[10.0, 0.0, 0.0], [0.0, 0.0, 3.0], [0.0, 2.0, 3.5]])
+    cfg = Cfg(3, 3, K=4, smooth=0.0)
+    rec = quantize(cfg, S)
+    assert list(rec.cid) == [0, 3 + 2, 2, 1]
+    np.testing.assert_array_equal(rec.cv[0], [10, 0, 0])
+    np.testing.assert_array_equal(rec.cv[1], [0, 3, 3.5])
+    np.testing.assert_array_equal(rec.cv[2], [0, 2, 0])
+    np.testing.assert_array_equal(rec.cv[3], [0, 0, 0])
+    assert np.all(rec.Q == 0)
+    np.testing.assert_array_equal(dequantize(cfg, rec), S)
+
+
+def test_selection_zero_state_and_index_ties():
+    cfg = Cfg(8, 8, K=4)
+    rec = quantize(cfg, np.zeros((8, 8)))
+    assert list(rec.cid) == [0, 1, 2, 3]
+    assert np.all(rec.cv == 0) and np.all(rec.Q == 0) and np.all(rec.sig == 1)
+    assert np.all(rec.m == 1)
+    # two equal rows: the lower index first; an equal column after both rows
+    S = np.zeros((8, 8))
+    S[5, 2] = S[2, 6] = 1.0
+    rec = quantize(Cfg(8, 8, K=2), S)
+    assert list(rec.cid) == [2, 5]
+
+
+def test_selection_picks_planted_lines_tiny_workload():
+    """Tiny GDN workload (seed 0): the 4 compensators are exactly the 2 planted
+    rows and the 2 planted columns."""
+    rng = np.random.default_rng(0)
+    S, rows, cols = wl.initial_states(rng, 1, 32, 32)
+    rec = quantize(Cfg(32, 32, K=4), S[0])
+    assert sorted(rec.cid) == sorted(list(rows[0]) + list(32 + cols[0]))
+
+
+def test_selection_picks_planted_lines_d128():
+    rng = np.random.default_rng(11)
+    S, rows, cols = wl.initial_states(rng, 6, 128, 128)
+    for t in range(6):
+        rec = quantize(Cfg(128, 128, K=4), S[t])
+        assert sorted(rec.cid) == sorted(list(rows[t]) + list(128 + cols[t]))
+
+
+def test_flush_partial_window_equals_fold():
+    """A flush after n < W tokens gives the same record as a window of length n."""
+    rng = np.random.default_rng(12)
+    dk = dv = 16
+    S0 = rng.standard_normal((dv, dk)) * 0.1
+    q, k, v, a, b = _inputs(rng, 5, dk, dv, 1)
+    t16 = Tile(Cfg(dk, dv, W=16, gate=1), S0)
+    t5 = Tile(Cfg(dk, dv, W=5, gate=1), S0)
+    o16 = t16.run(q, k, v, a, b)
+    o5 = t5.run(q, k, v, a, b)
+    t16.flush()
+    np.testing.assert_array_equal(o16, o5)
+    np.testing.assert_array_equal(t16.rec.Q, t5.rec.Q)
+    np.testing.assert_array_equal(t16.rec.cid, t5.rec.cid)
+
+
+# --------------------------------------------------------------------------
+# The pages' accounting
+# --------------------------------------------------------------------------
+
+def test_storage_accounting_matches_pages(golden_dir):
+    """int8 codes + per-row scales + per-column smoothing factors + 4 fp32
+    compensator lines (+ their ids) at d = 128: 1.19 bytes per value, 3.4x
+    below fp32, about 70 % less."""
+    g = json.load(open(os.path.join(golden_dir, "pages_accounting.json")))
+    cfg = Cfg(128, 128, W=g["window_tokens"], K=g["compensator_tokens"])
+    rec = quantize(cfg, np.random.default_rng(0).standard_normal((128, 128)))
+    nbytes = rec.Q.nbytes + rec.sig.nbytes + rec.m.nbytes + rec.cv.nbytes + rec.cid.nbytes
+    bpv = nbytes / (128 * 128)
+    assert round(bpv, 2) == g["bytes_per_value"]
+    assert round(g["fp32_bytes_per_value"] / bpv, 1) == g["reduction_vs_fp32"]
+    assert abs(100 * (1 - bpv / g["fp32_bytes_per_value"]) - g["storage_cut_percent_approx"]) < 1
+    assert wl.QWEN35_9B_GDN.window == g["window_tokens"]
+    assert wl.QWEN35_9B_GDN.n_comp == g["compensator_tokens"]
+    assert g["checkpoint_every_tokens"] % g["window_tokens"] == 0
+
+
+# --------------------------------------------------------------------------
+# Directional quality claims
+# --------------------------------------------------------------------------
+
+def _drift(cfg, S0, inp, o_ex):
+    tile = Tile(cfg, S0, wy_check=False)
+    o = tile.run(*inp)
+    num = np.linalg.norm(o - o_ex, axis=1)
+    return float(np.mean(num / np.linalg.norm(o_ex, axis=1)))
+
+
+def test_each_technique_reduces_drift():
+    """Per-window quantization, compensators and smoothing each lower the
+    output drift from the exact recurrence on the tiny GDN workload recipe."""
+    rng = np.random.default_rng(0)
+    d, T = 32, 256
+    S0, _, _ = wl.initial_states(rng, 1, d, d)
+    ti = wl.token_inputs(rng, wl.TINY_GDN, T)
+    inp = (ti.q[:, 0, 0], ti.k[:, 0, 0], ti.v[:, 0, 0], ti.alpha[:, 0, 0], ti.beta[:, 0, 0])
+    _, o_ex = exact_run(Cfg(d, d), S0[0], *inp)
+    full = _drift(Cfg(d, d, W=16, K=4, smooth=0.5), S0[0], inp, o_ex)
+    naive = _drift(Cfg(d, d, W=1, K=0, smooth=0.0), S0[0], inp, o_ex)
+    no_window = _drift(Cfg(d, d, W=1, K=4, smooth=0.5), S0[0], inp, o_ex)
+    no_comp = _drift(Cfg(d, d, W=16, K=0, smooth=0.5), S0[0], inp, o_ex)
+    assert full < 0.5 * naive
+    assert full < no_window
+    assert full < no_comp
+
+
+def test_batch_driver_matches_tile_runs():
+    """The OpenMP batch driver (CPU baseline) indexes grouped heads correctly."""
+    rng = np.random.default_rng(13)
+    w = wl.Workload("t", 2, 2, 4, 16, wl.GATE_DIAG, True, 20, window=4)
+    cfg = Cfg(16, 16, W=4, K=2, gate=1)
+    S0, _, _ = wl.initial_states(rng, w.tiles, 16, 16)
+    ti = wl.token_inputs(rng, w, 20)
+    tiles = [Tile(cfg, S0[t], wy_check=False) for t in range(w.tiles)]
+    rec = {"Q": np.stack([t.rec.Q for t in tiles]), "sig": np.stack([t.rec.sig for t in tiles]),
+           "m": np.stack([t.rec.m for t in tiles]), "cv": np.stack([t.rec.cv for t in tiles]),
+           "cid": np.stack([t.rec.cid for t in tiles])}
+    buf = {"n": np.zeros(w.tiles, np.int32), "bk": np.zeros((w.tiles, 4, 16)),
+           "bd": np.zeros((w.tiles, 4, 16)), "ba": np.zeros((w.tiles, 4, 16))}
+    inp = {n: np.ascontiguousarray(getattr(ti, n), dtype=np.float64)
+           for n in ("q", "k", "v", "alpha", "beta")}
+    inp["o"] = np.zeros((20, 2, 4, 16))
+    used = oracle.batch_run(cfg, 2, 2, 4, 20, rec, buf, inp, nthreads=2)
+    assert used >= 1
+    for t in range(w.tiles):
+        b, h = divmod(t, 4)
+        o = tiles[t].run(ti.q[:, b, h // 2], ti.k[:, b, h // 2], ti.v[:, b, h],
+                         ti.alpha[:, b, h], ti.beta[:, b, h])
+        np.testing.assert_array_equal(inp["o"][:, b, h], o)
+        np.testing.assert_array_equal(rec["Q"][t], tiles[t].rec.Q)
