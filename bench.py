@@ -1,0 +1,530 @@
+"""Benchmark of the int8-state LeapQuant GDN/KDA decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qwen35_9b_gdn|kimi_linear_kda] [--layers L]
+
+One step = one 16-token quantization window (15 plain decode tokens and the
+boundary token whose kernel also folds, compensates, smooths and requantizes)
+for every (sequence, value head) tile of L independent layer states, cycled
+token by token as a model's layers are.  The L states keep the working set far
+above the 126 MB L2, so every step streams its state from HBM.
+
+value = tile-steps/s (one tile-step = one decode token of one value head of
+one layer) with all inputs resident in HBM, timed with CUDA events around a
+CUDA-graph replay of K steps.  The same line carries: the in-house fp32-state
+kernel on the same workload and its speedup ratio, the roofline of the decode
+kernel against the measured HBM copy bandwidth, end-to-end throughput through
+the host-buffer C entry point, the CPU oracle timed on a sample, and the SM
+clocks sampled during the timed region.
+
+Multi-GPU (torchrun): every rank runs its own batch of sequences (weak
+scaling, no collective on the data path); time is the max over ranks.
+--impl reference times the CPU oracle (the reference arm) on host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from recurrent_state_quantization_decode_b200 import workloads as wl  # noqa: E402
+
+METRIC = ("decode tokens/s·head (int8 state) & achieved HBM GB/s vs 8 TB/s; "
+          "speedup vs fp32 state")
+UNIT = "tile-steps/s"
+NOMINAL_HBM_GBS = 8000.0
+WORKLOADS = {"qwen35_9b_gdn": wl.QWEN35_9B_GDN, "kimi_linear_kda": wl.KIMI_LINEAR_KDA}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_qwen35_9b_gdn.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "recurrent_state_quantization_decode_b200", "csrc", f)
+                  for f in ("lq_kernels.cu", "lq_internal.h")]
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic bytes (what the method must move, not what a kernel happens to)
+# ---------------------------------------------------------------------------
+
+def algorithmic_bytes_per_tile_step(w: wl.Workload, out_bytes: int = 4) -> dict:
+    """Average bytes one tile-step must move over a full window (token slots
+    n = 0..W-1).  Keys are shared by the Hv/Hk value heads of a key head, so
+    their bytes are divided among them."""
+    d, W, K = w.d, w.window, w.n_comp
+    inb = 2 if w.io_bf16 else 4
+    g = w.num_v_heads // w.num_k_heads
+    ga = d if w.gate == wl.GATE_DIAG else 1
+    record = d * d + 8 * d + 4 * K * d + 4 * K
+    record = (record + 15) // 16 * 16
+    entry = 4 * d + 4 * ga + inb * d / g          # d_i, alpha_i, k_i (shared)
+    mean_n = (W - 1) / 2.0
+    parts = {
+        "record_read": record,
+        "buffer_read": mean_n * entry,
+        "buffer_append": entry,
+        "fold_record_write": record / W,
+        "inputs": 2 * inb * d / g + inb * d + 4 * ga + 4,   # q, k (shared), v, alpha, beta
+        "output": out_bytes * d,
+        "phase_counter": 8,
+    }
+    parts["total"] = sum(parts.values())
+    return parts
+
+
+def fp32_bytes_per_tile_step(w: wl.Workload, out_bytes: int = 4) -> float:
+    d = w.d
+    inb = 2 if w.io_bf16 else 4
+    g = w.num_v_heads // w.num_k_heads
+    ga = d if w.gate == wl.GATE_DIAG else 1
+    return 2 * 4 * d * d + 2 * inb * d / g + inb * d + 4 * ga + 4 + out_bytes * d
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(tiles: int):
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary,
+    scaled to `tiles`; None if the summary is missing or the kernel source has
+    changed since it was captured."""
+    try:
+        txt = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
+    per_tile = re.search(r"dram_bytes_per_tile_step:\s*([0-9.]+)", txt)
+    if not sha or not per_tile or sha.group(1) != kernel_source_sha():
+        return None
+    return float(per_tile.group(1)) * tiles
+
+
+# ---------------------------------------------------------------------------
+# Clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def window(self, t0: float, t1: float) -> None:
+        """Keep only the samples taken between t0 and t1 (time.time())."""
+        self.t0, self.t1 = t0, t1
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        t0, t1 = getattr(self, "t0", 0.0), getattr(self, "t1", float("inf"))
+        for ts, ln in self.lines:
+            if ts < t0 or ts > t1:
+                continue
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+# ---------------------------------------------------------------------------
+
+def _oracle_inputs(w: wl.Workload, tiles_b: int, T: int, seed: int):
+    """Seeded inputs of `tiles_b` sequences (all heads) for T tokens, fp64."""
+    rng = np.random.default_rng(seed)
+    S0, _, _ = wl.initial_states(rng, tiles_b * w.num_v_heads, w.d, w.d)
+    ti = wl.token_inputs(rng, w, T, batch=tiles_b)
+    return S0, ti
+
+
+def run_oracle_sample(w: wl.Workload, seqs: int, seed: int = 1234) -> tuple[float, int, int]:
+    """Time the oracle on `seqs` sequences x all heads for one window
+    (init + W tokens incl. the fold).  Returns (seconds, tile_steps, threads)."""
+    import oracle
+
+    cfg = oracle.Cfg(w.d, w.d, W=w.window, K=w.n_comp, gate=w.gate, quant=1, smooth=w.smooth)
+    T = w.window
+    S0, ti = _oracle_inputs(w, seqs, T, seed)
+    tiles = seqs * w.num_v_heads
+    recs = [oracle.quantize(cfg, S0[t].astype(np.float64)) for t in range(tiles)]
+    rec = {"Q": np.stack([r.Q for r in recs]), "sig": np.stack([r.sig for r in recs]),
+           "m": np.stack([r.m for r in recs]), "cv": np.stack([r.cv for r in recs]),
+           "cid": np.stack([r.cid for r in recs])}
+    ga = w.d if w.gate == wl.GATE_DIAG else 1
+    buf = {"n": np.zeros(tiles, np.int32), "bk": np.zeros((tiles, w.window, w.d)),
+           "bd": np.zeros((tiles, w.window, w.d)), "ba": np.zeros((tiles, w.window, ga))}
+    inp = {n: np.ascontiguousarray(getattr(ti, n), dtype=np.float64)
+           for n in ("q", "k", "v", "alpha", "beta")}
+    inp["o"] = np.zeros((T, seqs, w.num_v_heads, w.d))
+    threads = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    used = oracle.batch_run(cfg, seqs, w.num_k_heads, w.num_v_heads, T, rec, buf, inp,
+                            nthreads=threads)
+    dt = time.perf_counter() - t0
+    return dt, tiles * T, used
+
+
+def calibrate_oracle_seqs(w: wl.Workload, target_s: float) -> int:
+    dt, ts, _ = run_oracle_sample(w, 1)
+    per_seq = max(dt, 1e-4)
+    return int(max(1, min(w.batch, math.floor(target_s / per_seq))))
+
+
+def cpu_baseline(w: wl.Workload, target_s: float = 15.0) -> dict:
+    seqs = calibrate_oracle_seqs(w, target_s)
+    dt, ts, used = run_oracle_sample(w, seqs)
+    return {"value": ts / dt, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": (f"{seqs} of {w.batch} sequences x {w.num_v_heads} heads, one "
+                       f"{w.window}-token window incl. the fold, one layer; fp64 C oracle, "
+                       f"OpenMP over tiles; {dt:.1f} s")}
+
+
+def reference_arm(args, w: wl.Workload, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    steps, warm = args.steps, args.warmup
+    budget = 150.0
+    dt1, ts1, _ = run_oracle_sample(w, 1)
+    seqs = int(max(1, min(w.batch, math.floor(budget / (steps + warm) / max(dt1, 1e-4)))))
+    for _ in range(warm):
+        run_oracle_sample(w, seqs)
+    tot_t, tot_ts, used = 0.0, 0, 1
+    for s in range(steps):
+        dt, ts, used = run_oracle_sample(w, seqs, seed=1234 + s)
+        tot_t += dt
+        tot_ts += ts
+    value = tot_ts / tot_t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": warm, "ms_per_step": 1e3 * tot_t / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, args.layers),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+                         "sample": (f"per step: {seqs} sequences x {w.num_v_heads} heads, one "
+                                    f"{w.window}-token window incl. the fold")},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w: wl.Workload, layers: int) -> dict:
+    return {"workload": w.name, "batch": w.batch, "num_k_heads": w.num_k_heads,
+            "num_v_heads": w.num_v_heads, "d_k": w.d, "d_v": w.d,
+            "gate": "scalar (GDN)" if w.gate == wl.GATE_SCALAR else "diagonal (KDA)",
+            "io": "bf16 q/k/v, fp32 o" if w.io_bf16 else "fp32", "window": w.window,
+            "compensators": w.n_comp, "smooth": w.smooth, "layers_cycled": layers,
+            "tiles_per_layer": w.tiles,
+            "step": f"one {w.window}-token window x {layers} layers",
+            "l2": "inputs larger than L2 (layer states cycled every token)"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+class Layer:
+    """One layer's stored state, fp32 comparison state and W tokens of inputs."""
+
+    def __init__(self, B, w: wl.Workload, seed: int, device):
+        import torch
+
+        rng = np.random.default_rng(seed)
+        S0, _, _ = wl.initial_states(rng, w.tiles, w.d, w.d)
+        ti = wl.token_inputs(rng, w, w.window)
+        dt = torch.bfloat16 if w.io_bf16 else torch.float32
+        self.cfg = B.config_for(w)
+        self.ds = B.DeviceState(self.cfg, device=device)
+        S0_dev = torch.from_numpy(S0).to(device)
+        B.lq_state_init(self.cfg, S0_dev, self.ds.st)
+        self.S32 = S0_dev  # the fp32-state path starts from the same states
+        self.q = torch.from_numpy(ti.q).to(device=device, dtype=dt)
+        self.k = torch.from_numpy(ti.k).to(device=device, dtype=dt)
+        self.v = torch.from_numpy(ti.v).to(device=device, dtype=dt)
+        self.alpha = torch.from_numpy(ti.alpha).to(device)
+        self.beta = torch.from_numpy(ti.beta).to(device)
+        self.out = torch.empty((w.batch, w.num_v_heads, w.d), dtype=torch.float32, device=device)
+        self.host = None
+
+    def pin_host_inputs(self):
+        import torch
+
+        self.host = {n: getattr(self, n).cpu().pin_memory()
+                     for n in ("q", "k", "v", "alpha", "beta")}
+        self.host_out = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        self.staging = torch.empty(self.ds.layout.host_staging_bytes, dtype=torch.uint8,
+                                   device=self.out.device)
+
+
+def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+
+    from recurrent_state_quantization_decode_b200 import binding as B
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    L = args.layers
+    layers = [Layer(B, w, seed=1000 * rank + l, device=device) for l in range(L)]
+    stream = torch.cuda.Stream(device=device)
+    W = w.window
+    launches_per_step = W * L
+
+    def step_int8(s):
+        for t in range(W):
+            for ly in layers:
+                B.lq_decode_step(ly.cfg, ly.q[t], ly.k[t], ly.v[t], ly.alpha[t], ly.beta[t],
+                                 ly.ds.st, ly.out, stream=s)
+
+    def step_fp32(s):
+        for t in range(W):
+            for ly in layers:
+                B.lq_fp32_decode_step(ly.cfg, ly.q[t], ly.k[t], ly.v[t], ly.alpha[t],
+                                      ly.beta[t], ly.S32, ly.out, stream=s)
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            fn(stream.cuda_stream)          # one eager pass (also warms up)
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                fn(stream.cuda_stream)
+        torch.cuda.synchronize()
+        return g
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(graph, steps, warmup, sample_clocks=False):
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                graph.replay()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        uuid = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            pass
+        sampler = ClockSampler(uuid if sample_clocks else None)
+        if sample_clocks:
+            sampler.__enter__()
+            time.sleep(0.3)
+        wall0 = time.time()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(steps):
+                graph.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        wall1 = time.time()
+        if sample_clocks:
+            time.sleep(0.15)
+            sampler.__exit__(None, None, None)
+            sampler.window(wall0, wall1)
+        barrier()
+        torch.cuda.synchronize()
+        ms = max_over_ranks(start.elapsed_time(end))
+        return ms, (sampler.summary() if sample_clocks else None)
+
+    g8 = capture(step_int8)
+    ms8, clocks = timed(g8, args.steps, args.warmup, sample_clocks=True)
+    err = max(B.lq_get_last_error(ly.ds.st, stream.cuda_stream) for ly in layers)
+    if err != B.LQ_OK:
+        raise RuntimeError(f"device error word set: {B.lq_status_string(err)}")
+    del g8
+    g32 = capture(step_fp32)
+    steps32 = max(3, args.steps // 4)
+    ms32, _ = timed(g32, steps32, args.warmup)
+    del g32
+
+    units_per_step = w.tiles * W * L               # per rank
+    value = world * units_per_step * args.steps / (ms8 / 1e3)
+    value32 = world * units_per_step * steps32 / (ms32 / 1e3)
+    ms_per_step = ms8 / args.steps
+
+    # roofline of the decode kernel (algorithmic bytes / graph time per launch)
+    ab = algorithmic_bytes_per_tile_step(w)
+    bytes_per_launch = ab["total"] * w.tiles
+    launch_s = (ms8 / 1e3) / (args.steps * launches_per_step)
+    achieved = bytes_per_launch / launch_s / 1e9
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    peak = float(peaks.get("hbm_gbs", 6650.0))
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    traffic = profiled_traffic(w.tiles)
+    fp32_bytes = fp32_bytes_per_tile_step(w) * w.tiles
+    fp32_achieved = fp32_bytes / ((ms32 / 1e3) / (steps32 * launches_per_step)) / 1e9
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        for ly in layers:
+            ly.pin_host_inputs()
+        h2d = sum(ly.host[n][0].numel() * ly.host[n][0].element_size()
+                  for ly in layers for n in ("q", "k", "v", "alpha", "beta")) * W
+        d2h = sum(ly.host_out.numel() * 4 for ly in layers) * W
+        e2e_steps = max(2, min(args.steps, 20))
+
+        def step_host(s):
+            for t in range(W):
+                for ly in layers:
+                    hs = ly.host
+                    B.lq_decode_step_host(ly.cfg, hs["q"][t], hs["k"][t], hs["v"][t],
+                                          hs["alpha"][t], hs["beta"][t], ly.ds.st,
+                                          ly.host_out, ly.staging, stream=s)
+
+        for _ in range(2):
+            step_host(stream.cuda_stream)
+        torch.cuda.synchronize()
+        barrier()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(e2e_steps):
+            step_host(stream.cuda_stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = max_over_ranks(start.elapsed_time(end))
+        e2e = {"value": world * units_per_step * e2e_steps / (ms_e2e / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "path": "lq_decode_step_host (pinned host q,k,v,alpha,beta in; o out)"}
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "state_dtype": "int8", "data": "synthetic", "config": workload_config(w, L),
+        "gpu_launches": args.steps * launches_per_step,
+        "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
+        "bytes_per_value": {"stored": ab["record_read"] / (w.d * w.d),
+                            "moved_per_step": ab["total"] / (w.d * w.d)},
+        "fp32_state": {"value": value32, "unit": UNIT, "ms_per_step": ms32 / steps32,
+                       "hbm_gbs": fp32_achieved, "steps": steps32},
+        "speedup_vs_fp32_state": value / value32,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": peak_src,
+                     "kernel": "decode_kernel<128,bf16,GDN> (int8 state)",
+                     "algorithmic_bytes_per_tile_step": ab["total"],
+                     "launch_time": "graph replay time / launches (includes inter-kernel gaps)"},
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen35_9b_gdn")
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, w, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        gpu_arm(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

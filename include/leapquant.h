@@ -1,0 +1,199 @@
+/*
+ * leapquant.h - C ABI of libleapquant.so: the per-token decode step of a
+ * Gated DeltaNet (GDN) / Kimi Delta Attention (KDA) layer whose recurrent
+ * state is stored in int8, following LeapQuant.
+ *
+ * Method sources (page title, section):
+ *  - "LeapQuant: Training-Free 8-bit Quantization for Linear Attention
+ *    Recurrent States" (zhichai.net forum summary), "Abstract (translated)",
+ *    items 1-3: per-window quantization (outputs from a fixed low-bit state
+ *    plus a high-precision buffer, quantize once at the window's end);
+ *    Compensator Tokens (largest outliers kept in high precision, sharing the
+ *    update path of real tokens); residual smoothing before quantization.
+ *  - "LeapQuant: Efficient Linear Attention with Accurate Recurrent State
+ *    Quantization" (opentrain.ai), "Abstract": the outliers are rows and
+ *    columns of the state; the FP32-state baseline.
+ *  - globaltechnewsdesk news article on LeapQuant, paragraphs 3-5: a window
+ *    of 16 tokens, reconstruct and quantize at the boundary, four
+ *    Compensator Tokens, 1.19 bytes per stored value, 4 bytes for FP32.
+ *
+ * Notation.  A tile is one (sequence b, value head h) state S, d x d, row i =
+ * value channel, column j = key channel, o = S q.  The exact recurrence is
+ *   S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ * with alpha_t a scalar (GDN) or a d-vector over key channels (KDA).
+ * Value head h reads key/query head h / (Hv / Hk).
+ *
+ * Stored state (caller-owned device memory, sizes from lq_state_layout):
+ *  records  [B*Hv] tile records, record_bytes each (a multiple of 16):
+ *           codes int8 [d][d] row-major | sigma fp32 [d] (per-row scale) |
+ *           m fp32 [d] (per-key-column smoothing factor) | compensator
+ *           vectors fp32 [K][d] | compensator ids int32 [K] (i = row i,
+ *           d + j = column j) | zero padding.  The window-base state is
+ *           S0_ij = sigma_i * code_ij * m_j plus the compensator lines.
+ *           At d = 128, K = 4 a record is 19,472 bytes = 1.19 bytes/value.
+ *  buf_k    [B][Hk][W][d] keys of the buffered tokens, in the input dtype
+ *           (lossless: they are the inputs themselves).
+ *  buf_d    [B][Hv][W][d] fp32 deltas d_i of the buffered tokens.
+ *  buf_g    [B][Hv][W] (GDN) or [B][Hv][W][d] (KDA) fp32 gates alpha_i.
+ *  buf_n    [B][Hv] int32 tokens buffered in the current window (0..W-1
+ *           between calls).
+ *  err      one int32 device error word (bit 0: a corrupt buf_n was seen).
+ * The layout is public: a checkpoint of a tile at a window boundary is a copy
+ * of its record.
+ *
+ * Conventions for every call:
+ *  - All pointers in lq_state and all tensor arguments are device pointers
+ *    unless the name says host; the library allocates nothing and keeps no
+ *    global state.  `stream` is a cudaStream_t (NULL = legacy default).
+ *  - Argument errors are detected on the host before anything is launched,
+ *    and reported synchronously: LQ_ERR_INVALID_ARG (null pointer, bad
+ *    shape), LQ_ERR_UNSUPPORTED (d not in {32, 64, 128}, W not in 1..16,
+ *    K not in 0..8, smooth not in {0, 0.5, 1}), LQ_ERR_MISALIGNED (records,
+ *    buffers or the fp32 state not 16-byte aligned).  A failed launch returns
+ *    LQ_ERR_CUDA.  Work is asynchronous on `stream`.
+ *  - Device-side problems never trap: a kernel sets a bit in *err and skips
+ *    the tile; lq_get_last_error reports it.
+ *  - batch == 0 is a valid empty call: nothing is launched.
+ *  - q is used as given (any 1/sqrt(d) scaling is the caller's).  NaN or Inf
+ *    inputs are outside the contract.
+ */
+#ifndef LEAPQUANT_H
+#define LEAPQUANT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LQ_OK = 0,
+  LQ_ERR_INVALID_ARG = 1,
+  LQ_ERR_UNSUPPORTED = 2,
+  LQ_ERR_MISALIGNED = 3,
+  LQ_ERR_CUDA = 4,
+  LQ_ERR_DEVICE_BOUNDS = 5
+} lq_status;
+
+typedef enum { LQ_GATE_SCALAR = 0, LQ_GATE_DIAG = 1 } lq_gate;
+typedef enum { LQ_DTYPE_F32 = 0, LQ_DTYPE_BF16 = 1 } lq_dtype;
+
+typedef struct {
+  int32_t batch;       /* B sequences (>= 0) */
+  int32_t num_k_heads; /* Hk >= 1 key/query heads */
+  int32_t num_v_heads; /* Hv >= 1 value heads, a multiple of Hk */
+  int32_t d;           /* d_k = d_v = d, one of 32, 64, 128 */
+  int32_t window;      /* W tokens per quantization window, 1..16 (16 on the pages) */
+  int32_t n_comp;      /* K compensator lines per tile, 0..8 (4 on the pages) */
+  int32_t gate;        /* lq_gate: LQ_GATE_SCALAR (GDN) or LQ_GATE_DIAG (KDA) */
+  int32_t in_dtype;    /* lq_dtype of q, k, v */
+  int32_t out_dtype;   /* lq_dtype of o */
+  float smooth;        /* smoothing exponent of the column max: 0, 0.5 or 1 */
+} lq_config;
+
+typedef struct {
+  size_t record_bytes;     /* one tile record, multiple of 16 */
+  size_t off_sigma;        /* byte offsets inside a record (codes start at 0) */
+  size_t off_m;
+  size_t off_comp_vec;
+  size_t off_comp_id;
+  size_t records_bytes;    /* B*Hv records */
+  size_t buf_k_bytes;
+  size_t buf_d_bytes;
+  size_t buf_g_bytes;
+  size_t buf_n_bytes;
+  size_t err_bytes;
+  size_t fp32_state_bytes; /* B*Hv*d*d*4: the unquantized comparison state */
+  size_t host_staging_bytes; /* device staging that lq_decode_step_host needs */
+} lq_layout;
+
+typedef struct {
+  void *records;
+  void *buf_k;
+  float *buf_d;
+  float *buf_g;
+  int32_t *buf_n;
+  int32_t *err;
+} lq_state;
+
+/* Interface version (1). */
+int32_t lq_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char *lq_status_string(lq_status s);
+
+/* Sizes and record offsets for cfg.  Host only; launches nothing. */
+lq_status lq_state_layout(const lq_config *cfg, lq_layout *out);
+
+/* Bytes of all stored state for cfg (records + buffers + counters + error
+ * word); *tile_bytes (nullable) receives one record's size and
+ * *buffer_bytes (nullable) the in-window buffers' total.  0 on a bad cfg. */
+size_t lq_state_bytes(const lq_config *cfg, size_t *tile_bytes, size_t *buffer_bytes);
+
+/* Quantize given fp32 states into records and empty the buffers (the
+ * "quantize the state" step of the zhichai.net summary's item 1, applied to a
+ * state produced elsewhere, e.g. by prefill).  S0: [B][Hv][d][d] fp32,
+ * 16-byte aligned.  mask: nullable [B] int32; sequences with mask[b] == 0 are
+ * left untouched.  Clears nothing else; the caller zeroes *err once. */
+lq_status lq_state_init(const lq_config *cfg, const float *S0, const lq_state *st,
+                        const int32_t *mask, void *stream);
+
+/* One decode token for every tile (zhichai.net summary, items 1-3; news
+ * article paragraph 3).  Reads the int8 record as stored (no dequantized copy
+ * in memory) and the buffered tokens, writes o_t = S_t q_t, appends
+ * (k_t, d_t, alpha_t) to the buffer, and when the buffer holds W tokens folds
+ * it into the state, extracts K compensator lines, smooths and requantizes
+ * the residual, all in the same kernel.
+ *  q, k  [B][Hk][d] in_dtype;  v [B][Hv][d] in_dtype;
+ *  alpha [B][Hv] (GDN) or [B][Hv][d] (KDA) fp32;  beta [B][Hv] fp32;
+ *  out   [B][Hv][d] out_dtype (written for active sequences only);
+ *  active nullable [B] int32: sequences with active[b] == 0 are skipped
+ *  entirely (state and output untouched). */
+lq_status lq_decode_step(const lq_config *cfg, const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta, const lq_state *st, void *out,
+                         const int32_t *active, void *stream);
+
+/* lq_decode_step with the token's inputs and output in HOST memory: copies
+ * q, k, v, alpha, beta to `staging` (device, layout.host_staging_bytes,
+ * 16-byte aligned), runs the step, and copies o back to out_host, all
+ * asynchronously on `stream` (the caller synchronizes before reading
+ * out_host; pinned host memory makes the copies truly asynchronous).  The
+ * state stays on the device.  active is a device pointer, as above. */
+lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const void *k_host,
+                              const void *v_host, const float *alpha_host,
+                              const float *beta_host, const lq_state *st, void *out_host,
+                              void *staging, const int32_t *active, void *stream);
+
+/* Fold a partially filled window now (0 < buf_n < W) for the selected
+ * sequences, exactly as the boundary fold does (news article, paragraph 3:
+ * reconstruct and quantize at the boundary).  Used at the end of a sequence
+ * or before taking a checkpoint off a boundary.  mask: nullable [B] int32. */
+lq_status lq_window_flush(const lq_config *cfg, const lq_state *st, const int32_t *mask,
+                          void *stream);
+
+/* The unquantized comparison path (the FP32-state baseline of the
+ * opentrain.ai abstract): S <- S diag(alpha); S <- S + beta (v - S k) k^T;
+ * o = S q, with S [B][Hv][d][d] fp32 read and written in place (16-byte
+ * aligned).  Other arguments as lq_decode_step. */
+lq_status lq_fp32_decode_step(const lq_config *cfg, const void *q, const void *k,
+                              const void *v, const float *alpha, const float *beta, float *S,
+                              void *out, void *stream);
+
+/* Materialize states as fp32 [B][Hv][d][d] (tests and drift reports):
+ * include_buffer == 0 gives the window-base state S0 of each record;
+ * include_buffer != 0 gives the current state, S0 advanced by the buffered
+ * tokens of the window. */
+lq_status lq_state_dequantize(const lq_config *cfg, const lq_state *st, int32_t include_buffer,
+                              float *S_out, void *stream);
+
+/* Synchronize `stream`, read and clear *err.  LQ_OK if no kernel reported a
+ * problem since the last call, LQ_ERR_DEVICE_BOUNDS otherwise, LQ_ERR_CUDA
+ * if the stream itself failed. */
+lq_status lq_get_last_error(const lq_state *st, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LEAPQUANT_H */

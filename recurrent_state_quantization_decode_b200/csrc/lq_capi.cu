@@ -1,0 +1,282 @@
+// C ABI of libleapquant.so (declared in include/leapquant.h): argument
+// validation on the host, then one kernel launch per call.  No call
+// allocates memory or keeps global state.
+
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "../../include/leapquant.h"
+#include "lq_internal.h"
+
+namespace {
+
+using lq::KParams;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t in_size(const lq_config *c) { return c->in_dtype == LQ_DTYPE_BF16 ? 2 : 4; }
+size_t out_size(const lq_config *c) { return c->out_dtype == LQ_DTYPE_BF16 ? 2 : 4; }
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Shape and option checks shared by every entry point.
+lq_status check_config(const lq_config *c) {
+  if (c == nullptr) return LQ_ERR_INVALID_ARG;
+  if (c->batch < 0 || c->num_k_heads < 1 || c->num_v_heads < 1) return LQ_ERR_INVALID_ARG;
+  if (c->num_v_heads % c->num_k_heads != 0) return LQ_ERR_INVALID_ARG;
+  if (c->gate != LQ_GATE_SCALAR && c->gate != LQ_GATE_DIAG) return LQ_ERR_INVALID_ARG;
+  if (c->in_dtype != LQ_DTYPE_F32 && c->in_dtype != LQ_DTYPE_BF16) return LQ_ERR_INVALID_ARG;
+  if (c->out_dtype != LQ_DTYPE_F32 && c->out_dtype != LQ_DTYPE_BF16) return LQ_ERR_INVALID_ARG;
+  if (c->d != 32 && c->d != 64 && c->d != 128) return LQ_ERR_UNSUPPORTED;
+  if (c->window < 1 || c->window > lq::kMaxWindow) return LQ_ERR_UNSUPPORTED;
+  if (c->n_comp < 0 || c->n_comp > lq::kMaxComp) return LQ_ERR_UNSUPPORTED;
+  if (!(c->smooth == 0.0f || c->smooth == 0.5f || c->smooth == 1.0f)) return LQ_ERR_UNSUPPORTED;
+  // grid.x is B * Hv CTAs
+  if (static_cast<int64_t>(c->batch) * c->num_v_heads > INT32_MAX) return LQ_ERR_UNSUPPORTED;
+  return LQ_OK;
+}
+
+lq_status check_state(const lq_config *c, const lq_state *st) {
+  if (st == nullptr) return LQ_ERR_INVALID_ARG;
+  if (!st->records || !st->buf_k || !st->buf_d || !st->buf_g || !st->buf_n || !st->err)
+    return LQ_ERR_INVALID_ARG;
+  if (!aligned16(st->records) || !aligned16(st->buf_k) || !aligned16(st->buf_d) ||
+      !aligned_to(st->buf_g, 4) || !aligned_to(st->buf_n, 4) || !aligned_to(st->err, 4))
+    return LQ_ERR_MISALIGNED;
+  (void)c;
+  return LQ_OK;
+}
+
+lq_status check_io(const lq_config *c, const void *q, const void *k, const void *v,
+                   const float *alpha, const float *beta, const void *out) {
+  if (!q || !k || !v || !alpha || !beta || !out) return LQ_ERR_INVALID_ARG;
+  const size_t is = in_size(c), os = out_size(c);
+  if (!aligned_to(q, is) || !aligned_to(k, is) || !aligned_to(v, is) || !aligned_to(alpha, 4) ||
+      !aligned_to(beta, 4) || !aligned_to(out, os))
+    return LQ_ERR_MISALIGNED;
+  return LQ_OK;
+}
+
+KParams make_params(const lq_config *c, const lq_state *st) {
+  KParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = c->batch;
+  p.Hk = c->num_k_heads;
+  p.Hv = c->num_v_heads;
+  p.d = c->d;
+  p.W = c->window;
+  p.K = c->n_comp;
+  p.gate = c->gate;
+  p.in_bf16 = c->in_dtype == LQ_DTYPE_BF16;
+  p.out_bf16 = c->out_dtype == LQ_DTYPE_BF16;
+  p.smooth = c->smooth == 0.0f ? 0 : (c->smooth == 0.5f ? 1 : 2);
+  p.L = lq::record_layout(c->d, c->n_comp);
+  if (st != nullptr) {
+    p.records = static_cast<uint8_t *>(st->records);
+    p.buf_k = st->buf_k;
+    p.buf_d = st->buf_d;
+    p.buf_g = st->buf_g;
+    p.buf_n = st->buf_n;
+    p.err = st->err;
+  }
+  return p;
+}
+
+lq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LQ_OK : LQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t lq_version(void) { return 1; }
+
+const char *lq_status_string(lq_status s) {
+  switch (s) {
+    case LQ_OK: return "LQ_OK";
+    case LQ_ERR_INVALID_ARG: return "LQ_ERR_INVALID_ARG: null pointer or bad shape";
+    case LQ_ERR_UNSUPPORTED: return "LQ_ERR_UNSUPPORTED: d, window, n_comp or smooth out of range";
+    case LQ_ERR_MISALIGNED: return "LQ_ERR_MISALIGNED: pointer not aligned as required";
+    case LQ_ERR_CUDA: return "LQ_ERR_CUDA: CUDA launch or stream error";
+    case LQ_ERR_DEVICE_BOUNDS: return "LQ_ERR_DEVICE_BOUNDS: a kernel found a corrupt window phase";
+  }
+  return "unknown lq_status";
+}
+
+lq_status lq_state_layout(const lq_config *cfg, lq_layout *out) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if (out == nullptr) return LQ_ERR_INVALID_ARG;
+  const lq::RecLayout L = lq::record_layout(cfg->d, cfg->n_comp);
+  const size_t B = cfg->batch, Hk = cfg->num_k_heads, Hv = cfg->num_v_heads;
+  const size_t d = cfg->d, W = cfg->window, tiles = B * Hv;
+  const size_t ga = cfg->gate == LQ_GATE_DIAG ? d : 1;
+  out->record_bytes = L.bytes;
+  out->off_sigma = L.off_sig;
+  out->off_m = L.off_m;
+  out->off_comp_vec = L.off_cv;
+  out->off_comp_id = L.off_cid;
+  out->records_bytes = tiles * L.bytes;
+  out->buf_k_bytes = B * Hk * W * d * in_size(cfg);
+  out->buf_d_bytes = tiles * W * d * 4;
+  out->buf_g_bytes = tiles * W * ga * 4;
+  out->buf_n_bytes = tiles * 4;
+  out->err_bytes = 4;
+  out->fp32_state_bytes = tiles * d * d * 4;
+  out->host_staging_bytes = 2 * round256(B * Hk * d * in_size(cfg)) +
+                            round256(tiles * d * in_size(cfg)) + round256(tiles * ga * 4) +
+                            round256(tiles * 4) + round256(tiles * d * out_size(cfg));
+  return LQ_OK;
+}
+
+size_t lq_state_bytes(const lq_config *cfg, size_t *tile_bytes, size_t *buffer_bytes) {
+  lq_layout L;
+  if (lq_state_layout(cfg, &L) != LQ_OK) return 0;
+  if (tile_bytes) *tile_bytes = L.record_bytes;
+  const size_t buffers = L.buf_k_bytes + L.buf_d_bytes + L.buf_g_bytes + L.buf_n_bytes;
+  if (buffer_bytes) *buffer_bytes = buffers;
+  return L.records_bytes + buffers + L.err_bytes;
+}
+
+lq_status lq_state_init(const lq_config *cfg, const float *S0, const lq_state *st,
+                        const int32_t *mask, void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if (S0 == nullptr) return LQ_ERR_INVALID_ARG;
+  if (!aligned16(S0) || !aligned_to(mask, 4)) return LQ_ERR_MISALIGNED;
+  if (cfg->batch == 0) return LQ_OK;
+  KParams p = make_params(cfg, st);
+  p.S_in = S0;
+  p.mask = mask;
+  return from_cuda(lq::launch_init(p, static_cast<cudaStream_t>(stream)));
+}
+
+lq_status lq_decode_step(const lq_config *cfg, const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta, const lq_state *st, void *out,
+                         const int32_t *active, void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if ((s = check_io(cfg, q, k, v, alpha, beta, out)) != LQ_OK) return s;
+  if (!aligned_to(active, 4)) return LQ_ERR_MISALIGNED;
+  if (cfg->batch == 0) return LQ_OK;
+  KParams p = make_params(cfg, st);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.out = out;
+  p.mask = active;
+  return from_cuda(lq::launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
+lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const void *k_host,
+                              const void *v_host, const float *alpha_host,
+                              const float *beta_host, const lq_state *st, void *out_host,
+                              void *staging, const int32_t *active, void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if ((s = check_io(cfg, q_host, k_host, v_host, alpha_host, beta_host, out_host)) != LQ_OK)
+    return s;
+  if (staging == nullptr) return LQ_ERR_INVALID_ARG;
+  if (!aligned16(staging) || !aligned_to(active, 4)) return LQ_ERR_MISALIGNED;
+  if (cfg->batch == 0) return LQ_OK;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const size_t B = cfg->batch, Hk = cfg->num_k_heads, Hv = cfg->num_v_heads, d = cfg->d;
+  const size_t tiles = B * Hv, ga = cfg->gate == LQ_GATE_DIAG ? d : 1;
+  const size_t nq = B * Hk * d * in_size(cfg), nv = tiles * d * in_size(cfg);
+  const size_t na = tiles * ga * 4, nb = tiles * 4, no = tiles * d * out_size(cfg);
+  uint8_t *base = static_cast<uint8_t *>(staging);
+  uint8_t *dq = base;
+  uint8_t *dk = dq + round256(nq);
+  uint8_t *dv = dk + round256(nq);
+  uint8_t *da = dv + round256(nv);
+  uint8_t *db = da + round256(na);
+  uint8_t *dout = db + round256(nb);
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(dq, q_host, nq, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dk, k_host, nq, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dv, v_host, nv, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(da, alpha_host, na, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(db, beta_host, nb, cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+    return LQ_ERR_CUDA;
+  KParams p = make_params(cfg, st);
+  p.q = dq;
+  p.k = dk;
+  p.v = dv;
+  p.alpha = reinterpret_cast<const float *>(da);
+  p.beta = reinterpret_cast<const float *>(db);
+  p.out = dout;
+  p.mask = active;
+  if ((e = lq::launch_decode(p, cs)) != cudaSuccess) return LQ_ERR_CUDA;
+  if ((e = cudaMemcpyAsync(out_host, dout, no, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+    return LQ_ERR_CUDA;
+  return LQ_OK;
+}
+
+lq_status lq_window_flush(const lq_config *cfg, const lq_state *st, const int32_t *mask,
+                          void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if (!aligned_to(mask, 4)) return LQ_ERR_MISALIGNED;
+  if (cfg->batch == 0) return LQ_OK;
+  KParams p = make_params(cfg, st);
+  p.mask = mask;
+  return from_cuda(lq::launch_flush(p, static_cast<cudaStream_t>(stream)));
+}
+
+lq_status lq_fp32_decode_step(const lq_config *cfg, const void *q, const void *k,
+                              const void *v, const float *alpha, const float *beta, float *S,
+                              void *out, void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_io(cfg, q, k, v, alpha, beta, out)) != LQ_OK) return s;
+  if (S == nullptr) return LQ_ERR_INVALID_ARG;
+  if (!aligned16(S)) return LQ_ERR_MISALIGNED;
+  if (cfg->batch == 0) return LQ_OK;
+  KParams p = make_params(cfg, nullptr);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.out = out;
+  return from_cuda(lq::launch_fp32_step(p, S, static_cast<cudaStream_t>(stream)));
+}
+
+lq_status lq_state_dequantize(const lq_config *cfg, const lq_state *st, int32_t include_buffer,
+                              float *S_out, void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if (S_out == nullptr) return LQ_ERR_INVALID_ARG;
+  if (!aligned16(S_out)) return LQ_ERR_MISALIGNED;
+  if (cfg->batch == 0) return LQ_OK;
+  KParams p = make_params(cfg, st);
+  p.S_out = S_out;
+  p.include_buffer = include_buffer != 0;
+  return from_cuda(lq::launch_dequantize(p, static_cast<cudaStream_t>(stream)));
+}
+
+lq_status lq_get_last_error(const lq_state *st, void *stream) {
+  if (st == nullptr || st->err == nullptr) return LQ_ERR_INVALID_ARG;
+  if (!aligned_to(st->err, 4)) return LQ_ERR_MISALIGNED;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  if (cudaMemcpyAsync(&word, st->err, sizeof(word), cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return LQ_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return LQ_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemsetAsync(st->err, 0, sizeof(int32_t), cs) != cudaSuccess) return LQ_ERR_CUDA;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return LQ_ERR_CUDA;
+    return LQ_ERR_DEVICE_BOUNDS;
+  }
+  return LQ_OK;
+}
+
+}  // extern "C"

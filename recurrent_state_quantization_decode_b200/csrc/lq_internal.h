@@ -1,0 +1,53 @@
+// Internal interface between the C ABI (lq_capi.cu) and the kernels
+// (lq_kernels.cu).  Not installed; callers use include/leapquant.h.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace lq {
+
+constexpr int kMaxWindow = 16;  // W limit: one buffer slot per token of a window
+constexpr int kMaxComp = 8;     // K limit
+constexpr int kErrBadPhase = 1;  // device error bit: buf_n outside [0, W)
+
+// Byte layout of one tile record (see include/leapquant.h).
+struct RecLayout {
+  int bytes;    // whole record, multiple of 16
+  int off_sig;  // fp32 [d]
+  int off_m;    // fp32 [d]
+  int off_cv;   // fp32 [K][d]
+  int off_cid;  // int32 [K]
+};
+
+RecLayout record_layout(int d, int K);
+
+// Everything a kernel launch needs; unused fields are null / zero.
+struct KParams {
+  int B, Hk, Hv, d, W, K, gate, in_bf16, out_bf16;
+  int smooth;  // 0: m = 1, 1: m = sqrt(colmax), 2: m = colmax
+  RecLayout L;
+  uint8_t *records;
+  void *buf_k;
+  float *buf_d;
+  float *buf_g;
+  int32_t *buf_n;
+  int32_t *err;
+  const void *q, *k, *v;
+  const float *alpha, *beta;
+  void *out;
+  const int32_t *mask;  // decode: active sequences; init / flush: selected sequences
+  const float *S_in;    // init: fp32 states to quantize
+  float *S_out;         // dequantize: fp32 states written
+  int include_buffer;   // dequantize: advance the base state by the buffered tokens
+};
+
+cudaError_t launch_decode(const KParams &p, cudaStream_t stream);
+cudaError_t launch_init(const KParams &p, cudaStream_t stream);
+cudaError_t launch_flush(const KParams &p, cudaStream_t stream);
+cudaError_t launch_dequantize(const KParams &p, cudaStream_t stream);
+cudaError_t launch_fp32_step(const KParams &p, float *S, cudaStream_t stream);
+
+}  // namespace lq
