@@ -73,7 +73,8 @@ typedef enum {
   LQ_ERR_UNSUPPORTED = 2,
   LQ_ERR_MISALIGNED = 3,
   LQ_ERR_CUDA = 4,
-  LQ_ERR_DEVICE_BOUNDS = 5
+  LQ_ERR_DEVICE_BOUNDS = 5,
+  LQ_ERR_TOO_LARGE = 6 /* lq_decode_step_host_noalloc: staging above its fixed array */
 } lq_status;
 
 typedef enum { LQ_GATE_SCALAR = 0, LQ_GATE_DIAG = 1 } lq_gate;
@@ -164,6 +165,34 @@ lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const vo
                               const void *v_host, const float *alpha_host,
                               const float *beta_host, const lq_state *st, void *out_host,
                               void *staging, const int32_t *active, void *stream);
+
+/* lq_decode_step_host for callers that cannot allocate device memory (the
+ * pages have no counterpart: this is an interface convenience).
+ *
+ * Some callers cannot call cudaMalloc: a plugin running inside a host
+ * application that owns every device allocation, or a latency-critical loop in
+ * which an allocation, which may synchronize the whole device, is not
+ * acceptable.  This variant takes no staging pointer: it stages the token's
+ * inputs and output in a fixed array of LQ_NOALLOC_STAGING_MAX_BYTES inside the
+ * library's own device memory, which every GPU that loads the library holds
+ * until the process exits.  It calls no allocating routine.
+ *  - Problems whose staging (layout.host_staging_bytes) exceeds
+ *    LQ_NOALLOC_STAGING_MAX_BYTES are rejected with LQ_ERR_TOO_LARGE before
+ *    anything is launched.
+ *  - All calls share the array and it keeps the previous call's contents; the
+ *    output region is cleared on every call, so outputs of inactive sequences
+ *    read back as zeros.  Calls that overlap on the GPU (other streams or other
+ *    threads) race on the array: the caller must order them.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ * Arguments and results are otherwise those of lq_decode_step_host. */
+#define LQ_NOALLOC_STAGING_MAX_BYTES ((size_t)8 << 20)
+lq_status lq_decode_step_host_noalloc(const lq_config *cfg, const void *q_host,
+                                      const void *k_host, const void *v_host,
+                                      const float *alpha_host, const float *beta_host,
+                                      const lq_state *st, void *out_host, const int32_t *active,
+                                      void *stream);
 
 /* Fold a partially filled window now (0 < buf_n < W) for the selected
  * sequences, exactly as the boundary fold does (news article, paragraph 3:

@@ -24,13 +24,15 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_MISALIGNED, LQ_ERR_CUDA, \
-    LQ_ERR_DEVICE_BOUNDS = range(6)
+    LQ_ERR_DEVICE_BOUNDS, LQ_ERR_TOO_LARGE = range(7)
+LQ_NOALLOC_STAGING_MAX_BYTES = 8 << 20  # the fixed staging array of the no-alloc entry point
 LQ_GATE_SCALAR, LQ_GATE_DIAG = 0, 1
 LQ_DTYPE_F32, LQ_DTYPE_BF16 = 0, 1
 
 # Every symbol include/leapquant.h declares.
 EXPORTED = ("lq_version", "lq_status_string", "lq_state_layout", "lq_state_bytes",
-            "lq_state_init", "lq_decode_step", "lq_decode_step_host", "lq_window_flush",
+            "lq_state_init", "lq_decode_step", "lq_decode_step_host",
+            "lq_decode_step_host_noalloc", "lq_window_flush",
             "lq_fp32_decode_step", "lq_state_dequantize", "lq_get_last_error")
 
 
@@ -67,6 +69,7 @@ _sig = {
     "lq_state_init": ([_CFG, _P, _ST, _P, _P], ctypes.c_int),
     "lq_decode_step": ([_CFG, _P, _P, _P, _P, _P, _ST, _P, _P, _P], ctypes.c_int),
     "lq_decode_step_host": ([_CFG, _P, _P, _P, _P, _P, _ST, _P, _P, _P, _P], ctypes.c_int),
+    "lq_decode_step_host_noalloc": ([_CFG, _P, _P, _P, _P, _P, _ST, _P, _P, _P], ctypes.c_int),
     "lq_window_flush": ([_CFG, _ST, _P, _P], ctypes.c_int),
     "lq_fp32_decode_step": ([_CFG, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "lq_state_dequantize": ([_CFG, _ST, ctypes.c_int32, _P, _P], ctypes.c_int),
@@ -174,6 +177,17 @@ def lq_decode_step_host(cfg, q_host, k_host, v_host, alpha_host, beta_host, stat
                                     _ptr(v_host), _ptr(alpha_host), _ptr(beta_host),
                                     ctypes.byref(state), _ptr(out_host), _ptr(staging),
                                     _ptr(active), _stream(stream)), "lq_decode_step_host")
+
+
+def lq_decode_step_host_noalloc(cfg, q_host, k_host, v_host, alpha_host, beta_host,
+                                state: lq_state, out_host, active=None, stream=None) -> None:
+    """lq_decode_step_host without a staging argument, for callers that cannot
+    allocate device memory: the library stages through its own fixed array of
+    LQ_NOALLOC_STAGING_MAX_BYTES (shared by all calls; overlapping calls race)."""
+    _check(_lib.lq_decode_step_host_noalloc(ctypes.byref(cfg), _ptr(q_host), _ptr(k_host),
+                                            _ptr(v_host), _ptr(alpha_host), _ptr(beta_host),
+                                            ctypes.byref(state), _ptr(out_host), _ptr(active),
+                                            _stream(stream)), "lq_decode_step_host_noalloc")
 
 
 def lq_window_flush(cfg, state: lq_state, mask=None, stream=None) -> None:

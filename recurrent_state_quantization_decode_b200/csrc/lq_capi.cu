@@ -100,6 +100,8 @@ const char *lq_status_string(lq_status s) {
     case LQ_ERR_MISALIGNED: return "LQ_ERR_MISALIGNED: pointer not aligned as required";
     case LQ_ERR_CUDA: return "LQ_ERR_CUDA: CUDA launch or stream error";
     case LQ_ERR_DEVICE_BOUNDS: return "LQ_ERR_DEVICE_BOUNDS: a kernel found a corrupt window phase";
+    case LQ_ERR_TOO_LARGE:
+      return "LQ_ERR_TOO_LARGE: staging exceeds the no-alloc entry point's fixed array";
   }
   return "unknown lq_status";
 }

@@ -27,7 +27,7 @@ def _declared():
 
 def test_exports_every_declared_symbol(B):
     names = _declared()
-    assert len(names) == 11
+    assert len(names) == 12
     assert sorted(B.EXPORTED) == names
     for n in names:
         assert hasattr(B._lib, n), n
@@ -106,5 +106,5 @@ def test_empty_batch_is_a_no_op(B):
 
 
 def test_status_strings(B):
-    for s in range(6):
+    for s in range(7):
         assert B.lq_status_string(s).startswith("LQ_")
