@@ -132,9 +132,9 @@ lq_status lq_state_layout(const lq_config *cfg, lq_layout *out);
  * *buffer_bytes (nullable) the in-window buffers' total.  0 on a bad cfg. */
 size_t lq_state_bytes(const lq_config *cfg, size_t *tile_bytes, size_t *buffer_bytes);
 
-/* Quantize given fp32 states into records and empty the buffers (the
- * "quantize the state" step of the zhichai.net summary's item 1, applied to a
- * state produced elsewhere, e.g. by prefill).  S0: [B][Hv][d][d] fp32,
+/* Quantize given fp32 states into records and empty the buffers: the same
+ * quantizer the window boundary runs (zhichai.net summary, items 1-3), applied
+ * to a state produced elsewhere, e.g. by prefill.  S0: [B][Hv][d][d] fp32,
  * 16-byte aligned.  mask: nullable [B] int32; sequences with mask[b] == 0 are
  * left untouched.  Clears nothing else; the caller zeroes *err once. */
 lq_status lq_state_init(const lq_config *cfg, const float *S0, const lq_state *st,
