@@ -50,7 +50,7 @@ NOMINAL_HBM_GBS = 8000.0
 WORKLOADS = {"qwen35_9b_gdn": wl.QWEN35_9B_GDN, "kimi_linear_kda": wl.KIMI_LINEAR_KDA}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_qwen35_9b_gdn.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "recurrent_state_quantization_decode_b200", "csrc", f)
-                  for f in ("lq_kernels.cu", "lq_internal.h")]
+                  for f in ("lq_decode.cu", "lq_internal.h")]
 
 
 # ---------------------------------------------------------------------------

@@ -34,10 +34,12 @@
  *  buf_k    [B][Hk][W][d] keys of the buffered tokens, in the input dtype
  *           (lossless: they are the inputs themselves).
  *  buf_d    [B][Hv][W][d] fp32 deltas d_i of the buffered tokens.
- *  buf_g    [B][Hv][W] (GDN) or [B][Hv][W][d] (KDA) fp32 gates alpha_i.
+ *  buf_g    [B][Hv][16] (GDN, the first W used) or [B][Hv][W][d] (KDA)
+ *           fp32 gates alpha_i.
  *  buf_n    [B][Hv] int32 tokens buffered in the current window (0..W-1
  *           between calls).
- *  err      one int32 device error word (bit 0: a corrupt buf_n was seen).
+ *  err      one int32 device error word (bit 0: a corrupt buf_n was seen;
+ *           bit 1: a bounded wait on a copy expired).
  * The layout is public: a checkpoint of a tile at a window boundary is a copy
  * of its record.
  *
@@ -52,7 +54,8 @@
  *    buffers or the fp32 state not 16-byte aligned).  A failed launch returns
  *    LQ_ERR_CUDA.  Work is asynchronous on `stream`.
  *  - Device-side problems never trap: a kernel sets a bit in *err and skips
- *    the tile; lq_get_last_error reports it.
+ *    the tile (or, when a wait on its own copy expires, stops after letting
+ *    its copies land); lq_get_last_error reports it.
  *  - batch == 0 is a valid empty call: nothing is launched.
  *  - q is used as given (any 1/sqrt(d) scaling is the caller's).  NaN or Inf
  *    inputs are outside the contract.
@@ -74,15 +77,16 @@ typedef enum {
   LQ_ERR_MISALIGNED = 3,
   LQ_ERR_CUDA = 4,
   LQ_ERR_DEVICE_BOUNDS = 5,
-  LQ_ERR_TOO_LARGE = 6 /* lq_decode_step_host_noalloc: staging above its fixed array */
+  LQ_ERR_TOO_LARGE = 6, /* lq_decode_step_host_noalloc: staging above its fixed array */
+  LQ_ERR_TIMEOUT = 7    /* a kernel's bounded wait on one of its copies expired */
 } lq_status;
 
 typedef enum { LQ_GATE_SCALAR = 0, LQ_GATE_DIAG = 1 } lq_gate;
 typedef enum { LQ_DTYPE_F32 = 0, LQ_DTYPE_BF16 = 1 } lq_dtype;
 
 typedef struct {
-  int32_t batch;       /* B sequences (>= 0) */
-  int32_t num_k_heads; /* Hk >= 1 key/query heads */
+  int32_t batch;       /* B sequences (0 <= B < 2^19) */
+  int32_t num_k_heads; /* Hk key/query heads, 1..2048 */
   int32_t num_v_heads; /* Hv >= 1 value heads, a multiple of Hk */
   int32_t d;           /* d_k = d_v = d, one of 32, 64, 128 */
   int32_t window;      /* W tokens per quantization window, 1..16 (16 on the pages) */
@@ -146,8 +150,9 @@ lq_status lq_state_init(const lq_config *cfg, const float *S0, const lq_state *s
  * (k_t, d_t, alpha_t) to the buffer, and when the buffer holds W tokens folds
  * it into the state, extracts K compensator lines, smooths and requantizes
  * the residual, all in the same kernel.
- *  q, k  [B][Hk][d] in_dtype;  v [B][Hv][d] in_dtype;
- *  alpha [B][Hv] (GDN) or [B][Hv][d] (KDA) fp32;  beta [B][Hv] fp32;
+ *  q, k  [B][Hk][d] in_dtype;  v [B][Hv][d] in_dtype (16-byte aligned);
+ *  alpha [B][Hv] (GDN) or [B][Hv][d] (KDA, 16-byte aligned) fp32;
+ *  beta  [B][Hv] fp32;
  *  out   [B][Hv][d] out_dtype (written for active sequences only);
  *  active nullable [B] int32: sequences with active[b] == 0 are skipped
  *  entirely (state and output untouched). */
@@ -217,8 +222,9 @@ lq_status lq_state_dequantize(const lq_config *cfg, const lq_state *st, int32_t 
                               float *S_out, void *stream);
 
 /* Synchronize `stream`, read and clear *err.  LQ_OK if no kernel reported a
- * problem since the last call, LQ_ERR_DEVICE_BOUNDS otherwise, LQ_ERR_CUDA
- * if the stream itself failed. */
+ * problem since the last call; LQ_ERR_TIMEOUT if a bounded wait expired;
+ * LQ_ERR_DEVICE_BOUNDS if a corrupt window phase was seen; LQ_ERR_CUDA if the
+ * stream itself failed. */
 lq_status lq_get_last_error(const lq_state *st, void *stream);
 
 #ifdef __cplusplus

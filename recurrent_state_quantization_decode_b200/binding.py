@@ -24,7 +24,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_MISALIGNED, LQ_ERR_CUDA, \
-    LQ_ERR_DEVICE_BOUNDS, LQ_ERR_TOO_LARGE = range(7)
+    LQ_ERR_DEVICE_BOUNDS, LQ_ERR_TOO_LARGE, LQ_ERR_TIMEOUT = range(8)
 LQ_NOALLOC_STAGING_MAX_BYTES = 8 << 20  # the fixed staging array of the no-alloc entry point
 LQ_GATE_SCALAR, LQ_GATE_DIAG = 0, 1
 LQ_DTYPE_F32, LQ_DTYPE_BF16 = 0, 1

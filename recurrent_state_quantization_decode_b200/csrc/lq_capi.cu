@@ -33,8 +33,10 @@ lq_status check_config(const lq_config *c) {
   if (c->window < 1 || c->window > lq::kMaxWindow) return LQ_ERR_UNSUPPORTED;
   if (c->n_comp < 0 || c->n_comp > lq::kMaxComp) return LQ_ERR_UNSUPPORTED;
   if (!(c->smooth == 0.0f || c->smooth == 0.5f || c->smooth == 1.0f)) return LQ_ERR_UNSUPPORTED;
-  // grid.x is B * Hv CTAs
+  // tiles are indexed with 32-bit ints; the decode kernel packs (sequence,
+  // key head) of a tile into one int
   if (static_cast<int64_t>(c->batch) * c->num_v_heads > INT32_MAX) return LQ_ERR_UNSUPPORTED;
+  if (c->batch >= (1 << 19) || c->num_k_heads > 2048) return LQ_ERR_UNSUPPORTED;
   return LQ_OK;
 }
 
@@ -49,11 +51,13 @@ lq_status check_state(const lq_config *c, const lq_state *st) {
   return LQ_OK;
 }
 
+// q, k, v (and the KDA gate) are moved with 16-byte bulk copies.
 lq_status check_io(const lq_config *c, const void *q, const void *k, const void *v,
                    const float *alpha, const float *beta, const void *out) {
   if (!q || !k || !v || !alpha || !beta || !out) return LQ_ERR_INVALID_ARG;
-  const size_t is = in_size(c), os = out_size(c);
-  if (!aligned_to(q, is) || !aligned_to(k, is) || !aligned_to(v, is) || !aligned_to(alpha, 4) ||
+  const size_t os = out_size(c);
+  const size_t as = c->gate == LQ_GATE_DIAG ? 16 : 4;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned_to(alpha, as) ||
       !aligned_to(beta, 4) || !aligned_to(out, os))
     return LQ_ERR_MISALIGNED;
   return LQ_OK;
@@ -102,6 +106,7 @@ const char *lq_status_string(lq_status s) {
     case LQ_ERR_DEVICE_BOUNDS: return "LQ_ERR_DEVICE_BOUNDS: a kernel found a corrupt window phase";
     case LQ_ERR_TOO_LARGE:
       return "LQ_ERR_TOO_LARGE: staging exceeds the no-alloc entry point's fixed array";
+    case LQ_ERR_TIMEOUT: return "LQ_ERR_TIMEOUT: a kernel's bounded wait on a copy expired";
   }
   return "unknown lq_status";
 }
@@ -122,7 +127,7 @@ lq_status lq_state_layout(const lq_config *cfg, lq_layout *out) {
   out->records_bytes = tiles * L.bytes;
   out->buf_k_bytes = B * Hk * W * d * in_size(cfg);
   out->buf_d_bytes = tiles * W * d * 4;
-  out->buf_g_bytes = tiles * W * ga * 4;
+  out->buf_g_bytes = cfg->gate == LQ_GATE_DIAG ? tiles * W * d * 4 : tiles * lq::kGdnGateStride * 4;
   out->buf_n_bytes = tiles * 4;
   out->err_bytes = 4;
   out->fp32_state_bytes = tiles * d * d * 4;
@@ -276,7 +281,7 @@ lq_status lq_get_last_error(const lq_state *st, void *stream) {
   if (word != 0) {
     if (cudaMemsetAsync(st->err, 0, sizeof(int32_t), cs) != cudaSuccess) return LQ_ERR_CUDA;
     if (cudaStreamSynchronize(cs) != cudaSuccess) return LQ_ERR_CUDA;
-    return LQ_ERR_DEVICE_BOUNDS;
+    return (word & lq::kErrTimeout) ? LQ_ERR_TIMEOUT : LQ_ERR_DEVICE_BOUNDS;
   }
   return LQ_OK;
 }

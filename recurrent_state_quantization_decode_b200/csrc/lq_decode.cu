@@ -1,0 +1,1640 @@
+// Kernels of the int8-state LeapQuant GDN/KDA decode step for sm_100a.
+//
+// Method (page title, section): zhichai.net summary "LeapQuant: Training-Free
+// 8-bit Quantization for Linear Attention Recurrent States", "Abstract
+// (translated)" items 1-3; opentrain.ai "LeapQuant: Efficient Linear Attention
+// with Accurate Recurrent State Quantization", "Abstract"; globaltechnewsdesk
+// news article on LeapQuant, paragraphs 3-5.  A tile (sequence, value head)
+// keeps a window-base state S0 = diag(sigma) Q diag(m) + compensator lines in
+// int8 for a window of W tokens; each token's output comes from S0 plus the
+// buffered tokens of the window, and the W-th token folds the buffer and
+// requantizes.
+//
+// Design for B200:
+//  * decode_kernel is persistent: about two CTAs per SM, each walking its tiles
+//    through a shared-memory ring of two or three slots (three where they fit
+//    in half an SM's shared memory).  One thread moves a tile's record (int8
+//    codes + scales + lines), its buffered tokens and its inputs with bulk
+//    asynchronous copies (cp.async.bulk, one destination CTA) that complete on
+//    an mbarrier, so the next tiles stream in while the current one is computed.
+//    Every mbarrier wait is bounded; on expiry the kernel flags the error word,
+//    drains its own copies and returns.
+//  * The two products y_q = S0 (Gamma o q) and y_k = S0 (Gamma o k) run on the
+//    int8 tensor path: the stored codes are the A operand as they are, and the
+//    two fp32 vectors x = m o Gamma o {q, k} are split exactly into four
+//    radix-128 int8 digits each (8 columns = one n8 tile) with a power-of-two
+//    scale.  The integer dot products are exact, so the result is the fp32
+//    product up to the digits' truncation (<= 7.5e-9 max|x| per element) and
+//    one rounding per combination step.  No code is ever converted to float on
+//    this path.
+//  * GDN with bf16 inputs takes a shorter per-token path: one warp does all
+//    per-channel work (gate product, x, digits, compensator dots) with no CTA
+//    barrier between the max and the digits, one warp gets the buffer
+//    coefficients c_s = rho_s k_s . k and a_s = rho_s k_s . q from a bf16
+//    m16n8k16 product, and the other row warps fetch their codes meanwhile.
+//  * On the boundary token the fp32 state S = S0 diag(Gamma) + sum d_s kt_s^T
+//    is built in registers, in the same fragment layout as the codes, and the
+//    quantizer (compensator lines, smoothing, per-row int8) runs on it.
+//
+// Fragment layout: warp w < D/16 owns state rows 16w..16w+15; lane (g = lane/4,
+// t = lane%4) owns rows 16w+g and 16w+g+8 and, in every 64-column span h, the
+// 16 columns 64h + 16t .. 64h + 16t + 15 (for d = 32 only t < 2 hold columns).
+//
+// Quantizer decisions use correctly rounded fp32 operations and fp64 line
+// energies, so a given fp32 state always yields the same record.
+
+#include <cfloat>
+#include <cstdint>
+#include <type_traits>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "lq_internal.h"
+
+namespace lq {
+
+RecLayout record_layout(int d, int K) {
+  RecLayout L;
+  L.off_sig = d * d;
+  L.off_m = L.off_sig + 4 * d;
+  L.off_cv = L.off_m + 4 * d;
+  L.off_cid = L.off_cv + 4 * K * d;
+  L.bytes = (L.off_cid + 4 * K + 15) / 16 * 16;
+  return L;
+}
+
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxTilesPerCta = 128;
+constexpr uint32_t kWaitLimit = 1u << 24;
+
+// ---------------------------------------------------------------------------
+// Geometry and shared-memory layout
+// ---------------------------------------------------------------------------
+
+template <int D>
+struct FG {
+  static constexpr int NRB = D / 16;                  // warps that own state rows
+  static constexpr int NSPAN = D >= 64 ? D / 64 : 1;  // 64-column spans
+  static constexpr int PADW = D + D / 4;              // padded column vectors
+  static constexpr int DIGW = 192;                    // digit row stride in bytes
+  static_assert(NRB <= kWarps, "one warp per 16 rows");
+};
+
+// Padded index of column j: 4 floats of padding after every 16, so that the
+// 16-float chunks that a warp reads start in different bank groups.
+__device__ __forceinline__ int padc(int j) { return j + ((j >> 4) << 2); }
+__device__ __forceinline__ int frag_col(int h, int t, int e) { return 64 * h + 16 * t + e; }
+template <int D>
+__device__ __forceinline__ bool chunk_valid(int t) {
+  return D >= 64 || 16 * t < D;
+}
+
+// One tile's staged data (a ring slot): the record, the buffered tokens and the
+// token's inputs, each at a 16-byte aligned offset.  The record area has the
+// record's actual size (it depends on K).
+template <int D, bool BF16, bool KDA>
+struct SL {
+  static constexpr int IB = BF16 ? 2 : 4;
+  static constexpr int BD = kMaxWindow * D * 4;                  // fp32 [W][D]
+  static constexpr int BK = kMaxWindow * D * IB;                 // in dtype [W][D]
+  static constexpr int BG = KDA ? kMaxWindow * D * 4 : kGdnGateStride * 4;
+  static constexpr int TAIL = BD + BK + BG + 3 * D * IB + (KDA ? D * 4 : 0);
+  // quantizer scratch aliased over the codes once they are in registers
+  static constexpr int QS_COLPART = 0;                           // fp64 [D/16][D]
+  static constexpr int QS_COLMAX = FG<D>::NRB * D * 8;           // fp32 [D/16][D]
+  static_assert(QS_COLMAX + FG<D>::NRB * D * 4 <= D * D, "scratch fits over the codes");
+  int bd, bk, bg, q, k, v, a, bytes;
+  __host__ __device__ explicit SL(int rec_bytes) {
+    bd = rec_bytes;
+    bk = bd + BD;
+    bg = bk + BK;
+    q = bg + BG;
+    k = q + D * IB;
+    v = k + D * IB;
+    a = v + D * IB;
+    bytes = (rec_bytes + TAIL + 127) / 128 * 128;
+  }
+};
+
+// Decode kernel variants.  GDN with bf16 inputs computes the buffer
+// coefficients on the bf16 tensor path (fast) and, at d = 128, keeps the
+// fold's scaled keys over the staged codes instead of in the scratch, which
+// leaves room for three ring slots at two CTAs per SM.
+template <int D, bool BF16, bool KDA>
+struct DecodeTraits {
+  static constexpr bool kFast = BF16 && !KDA;
+  static constexpr bool kKtOverCodes = kFast && kMaxWindow * FG<D>::PADW * 4 <= D * D;
+  static constexpr int kStages = kFast ? 3 : 2;
+};
+
+// The scaled-key array lives in the scratch unless the decode kernel keeps it
+// over the staged codes (GDN with bf16 inputs).
+template <int D, bool KT>
+struct KtArea {
+  alignas(16) float kt[kMaxWindow][FG<D>::PADW];  // keys times decay ratio to the last token
+};
+template <int D>
+struct KtArea<D, false> {};
+
+template <int D, bool KT>
+struct Scratch : KtArea<D, KT> {
+  alignas(16) float qf[D];
+  alignas(16) float kf[D];
+  alignas(16) float vf[D];
+  alignas(16) float G[D];                          // window gate Gamma per key channel
+  alignas(16) float mG[FG<D>::PADW];               // m o Gamma
+  alignas(16) float invm[FG<D>::PADW];             // 1 / m (new smoothing factors)
+  alignas(16) int8_t dig[8][FG<D>::DIGW];          // digits: rows 0-3 of x_q, 4-7 of x_k
+  alignas(16) float yq[D];
+  alignas(16) float yk[D];
+  alignas(16) float line[D];                       // the compensator line being extracted
+  alignas(16) double rowE[D];
+  float cc[kMaxWindow + 1];
+  float aa[kMaxWindow + 1];
+  float cpart[kMaxComp][kWarps][2];  // per-warp partial row-compensator dots
+  float rho[kMaxWindow + 1];         // scalar decay ratios (GDN)
+  double pbest[kWarps];              // per-warp partial argmax of the line energies
+  int pid[kWarps];
+  float xmax[2][kWarps];
+  float xscale[2];
+  int abort;
+  int warp_cnt[kWarps];
+  int tl_tile[kMaxTilesPerCta];
+  int tl_n[kMaxTilesPerCta];      // window phase; -1: skip (corrupt phase)
+  int tl_coord[kMaxTilesPerCta];  // b << 12 | hk << 1 | (this value head writes the key)
+  float tl_a[kMaxTilesPerCta];
+  float tl_b[kMaxTilesPerCta];
+  alignas(8) unsigned long long bar[3];
+};
+
+// ---------------------------------------------------------------------------
+// Small helpers and PTX wrappers
+// ---------------------------------------------------------------------------
+
+template <bool BF16>
+using in_t = std::conditional_t<BF16, __nv_bfloat16, float>;
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ void st_out(void *p, size_t i, float x, int bf16) {
+  if (bf16)
+    reinterpret_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(x);
+  else
+    reinterpret_cast<float *>(p)[i] = x;
+}
+
+__device__ __forceinline__ void load16(const float *src, float (&dst)[16]) {
+  const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float4 v = s4[u];
+    dst[4 * u] = v.x;
+    dst[4 * u + 1] = v.y;
+    dst[4 * u + 2] = v.z;
+    dst[4 * u + 3] = v.w;
+  }
+}
+
+// int8 code e (0..15) of a 16-byte chunk as a float, without an int->float
+// conversion: the byte, biased to unsigned, becomes the low mantissa byte of
+// 2^23 + (c + 128), and subtracting 2^23 + 128 recovers c exactly.
+__device__ __forceinline__ float code_at(const uint4 &c, int e) {
+  const uint32_t w = (e < 4) ? c.x : (e < 8) ? c.y : (e < 12) ? c.z : c.w;
+  const uint32_t bits = __byte_perm(w ^ 0x80808080u, 0x4B000000u, 0x7540u + (e & 3));
+  return __uint_as_float(bits) - 8388736.0f;
+}
+
+// Round-half-even of |x| < 2^22 with one add: the integer lands in the low
+// mantissa bits of x + 1.5 * 2^23 (its low byte is the two's-complement int8).
+constexpr float kRoundMagic = 12582912.0f;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *ptr) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long *bar, uint32_t bytes) {
+  unsigned long long state;
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 %0, [%1], %2;"
+               : "=l"(state)
+               : "r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+  (void)state;
+}
+
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long *bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on one phase of an mbarrier; false after kWaitLimit polls.
+__device__ __forceinline__ bool mbar_wait_bounded(unsigned long long *bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kWaitLimit; ++it)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// Global -> shared bulk copy into this CTA only, completing on `bar`.  dst, src and
+// bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         unsigned long long *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before the
+// async-proxy writes of a following bulk copy into the same memory.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// D (16x8, int32) += A (16x32, int8, row) x B (32x8, int8, col).
+__device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                       uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D (16x8, fp32) += A (16x16, bf16, row) x B (16x8, bf16, col).
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Exact split of x into four radix-128 digits with the power-of-two scale
+// s = 2^(E-6), where max|x| = M < 2^E:  x = s (d0 + d1/128 + d2/128^2 +
+// d3/128^3) + r with |r| <= s / (2 * 128^3).  Every step is exact in fp32,
+// and |d_i| <= 64.
+__device__ __forceinline__ void split_digits(float x, float M, int8_t *dst, int stride) {
+  int8_t d[4] = {0, 0, 0, 0};
+  if (M > 0.0f) {
+    const int eb = static_cast<int>((__float_as_uint(M) >> 23) & 0xffu);
+    float u;
+    if (eb >= 6) {
+      // M < 2^(eb - 126): multiply by 2^(132 - eb), exact
+      u = x * __uint_as_float(static_cast<uint32_t>(259 - eb) << 23);
+    } else {
+      int E;
+      frexpf(M, &E);
+      u = ldexpf(x, 6 - E);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float biased = u + kRoundMagic;
+      d[i] = static_cast<int8_t>(__float_as_uint(biased) & 0xffu);
+      u = (u - (biased - kRoundMagic)) * 128.0f;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i * stride] = d[i];
+}
+
+// max over the warp of |x| (one redux instruction on sm_100a)
+__device__ __forceinline__ float warp_max_abs(float x) {
+  float r;
+  asm volatile("redux.sync.max.abs.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// Sums 8 per-lane values over the warp: afterwards every lane holds the total
+// of value (lane >> 2) & 7.
+__device__ __forceinline__ float warp_sum8(float (&v)[8], int lane) {
+#pragma unroll
+  for (int step = 16, half = 4; step >= 4; step >>= 1, half >>= 1) {
+    const bool upper = (lane & step) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(kFull, send, step);
+    }
+  }
+  float r = v[0];
+  r += __shfl_xor_sync(kFull, r, 2);
+  r += __shfl_xor_sync(kFull, r, 1);
+  return r;
+}
+
+__device__ __forceinline__ float digit_scale(float M) {
+  if (!(M > 0.0f)) return 0.0f;
+  int E;
+  frexpf(M, &E);
+  return ldexpf(1.0f, E - 6);
+}
+
+// Reduce NV per-lane values over the 8 lanes that share t (lane bits 2-4),
+// halving the set at each step: afterwards lane (g, t) holds the totals of
+// values NV/8 * g .. NV/8 * g + NV/8 - 1 in v[0 .. NV/8) (for NV = 16:
+// values 2g and 2g + 1).
+template <int NV, typename T, typename Op>
+__device__ __forceinline__ void butterfly_g(T (&v)[NV], int lane, Op op) {
+#pragma unroll
+  for (int step = 16, half = NV / 2; step >= 4; step >>= 1, half >>= 1) {
+    const bool upper = (lane & step) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const T send = upper ? v[i] : v[i + half];
+      const T keep = upper ? v[i + half] : v[i];
+      v[i] = op(keep, __shfl_xor_sync(kFull, send, step));
+    }
+  }
+}
+
+struct AddOp {
+  template <typename T>
+  __device__ __forceinline__ T operator()(T a, T b) const { return a + b; }
+};
+struct MaxOp {
+  __device__ __forceinline__ float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+
+// ---------------------------------------------------------------------------
+// State build and quantizer (fragment layout)
+// ---------------------------------------------------------------------------
+
+// Loads the thread's codes (rows r0 = 16 warp + g and r0 + 8, its 16-byte
+// chunk of every span) from the staged record.
+template <int D>
+__device__ __forceinline__ void load_codes(const uint8_t *codes, uint4 (&A)[2][FG<D>::NSPAN]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int r0 = 16 * warp + g;
+#pragma unroll
+  for (int h = 0; h < FG<D>::NSPAN; ++h) {
+    if (chunk_valid<D>(t)) {
+      A[0][h] = *reinterpret_cast<const uint4 *>(codes + r0 * D + frag_col(h, t, 0));
+      A[1][h] = *reinterpret_cast<const uint4 *>(codes + (r0 + 8) * D + frag_col(h, t, 0));
+    } else {
+      A[0][h] = make_uint4(0, 0, 0, 0);
+      A[1][h] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+// Element e (0..15) of span h of row rr in a float2 register tile.
+#define SX(rr, h, e) ((((e) & 1) != 0) ? S[rr][h][(e) >> 1].y : S[rr][h][(e) >> 1].x)
+
+// The fp32 state of the thread's block (warps that own rows), as float2 pairs
+// along the columns:
+//   S_ij = sigma_i code_ij (m_j Gamma_j) + sum_{s < nent} d_s[i] kt_s[j]
+//          + Gamma_j * (compensator lines),
+// with kt_s = k_s o (decay ratio to the last token) in kt (rows of PADW) and m o Gamma in
+// s.mG.  rsig, rcv, rcid point at the staged record; bd at the staged deltas.
+template <int D, class SC>
+__device__ __forceinline__ void build_state(const SC &s, const float *kt,
+                                            const uint4 (&A)[2][FG<D>::NSPAN],
+                                            const float *rsig, const float *rcv, const int *rcid,
+                                            const float *bd, int nent, int K,
+                                            float2 (&S)[2][FG<D>::NSPAN][8]) {
+  using G = FG<D>;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int r0 = 16 * warp + g, r1 = r0 + 8;
+  const float2 sg0 = make_float2(rsig[r0], rsig[r0]), sg1 = make_float2(rsig[r1], rsig[r1]);
+#pragma unroll
+  for (int h = 0; h < G::NSPAN; ++h) {
+    if (chunk_valid<D>(t)) {
+      const float4 *mg4 = reinterpret_cast<const float4 *>(&s.mG[padc(frag_col(h, t, 0))]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 m = mg4[u];
+        const float2 ma = make_float2(m.x, m.y), mb = make_float2(m.z, m.w);
+        const int e = 4 * u;
+        S[0][h][2 * u] = __fmul2_rn(__fmul2_rn(sg0, make_float2(code_at(A[0][h], e),
+                                                                 code_at(A[0][h], e + 1))), ma);
+        S[0][h][2 * u + 1] = __fmul2_rn(
+            __fmul2_rn(sg0, make_float2(code_at(A[0][h], e + 2), code_at(A[0][h], e + 3))), mb);
+        S[1][h][2 * u] = __fmul2_rn(__fmul2_rn(sg1, make_float2(code_at(A[1][h], e),
+                                                                 code_at(A[1][h], e + 1))), ma);
+        S[1][h][2 * u + 1] = __fmul2_rn(
+            __fmul2_rn(sg1, make_float2(code_at(A[1][h], e + 2), code_at(A[1][h], e + 3))), mb);
+      }
+    } else {
+#pragma unroll
+      for (int e2 = 0; e2 < 8; ++e2) S[0][h][e2] = S[1][h][e2] = make_float2(0.0f, 0.0f);
+    }
+  }
+  // rank-nent update, two columns per packed FMA
+  for (int sl = 0; sl < nent; ++sl) {
+    const float2 d0 = make_float2(bd[sl * D + r0], bd[sl * D + r0]);
+    const float2 d1 = make_float2(bd[sl * D + r1], bd[sl * D + r1]);
+#pragma unroll
+    for (int h = 0; h < G::NSPAN; ++h) {
+      if (!chunk_valid<D>(t)) continue;
+      const float4 *k4 =
+          reinterpret_cast<const float4 *>(&kt[sl * G::PADW + padc(frag_col(h, t, 0))]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 k = k4[u];
+        const float2 ka = make_float2(k.x, k.y), kb = make_float2(k.z, k.w);
+        S[0][h][2 * u] = __ffma2_rn(d0, ka, S[0][h][2 * u]);
+        S[0][h][2 * u + 1] = __ffma2_rn(d0, kb, S[0][h][2 * u + 1]);
+        S[1][h][2 * u] = __ffma2_rn(d1, ka, S[1][h][2 * u]);
+        S[1][h][2 * u + 1] = __ffma2_rn(d1, kb, S[1][h][2 * u + 1]);
+      }
+    }
+  }
+  // compensator lines, decayed by Gamma
+  for (int c = 0; c < K; ++c) {
+    const int id = rcid[c];
+    if (id < D) {
+      if ((id == r0 || id == r1) && chunk_valid<D>(t)) {
+        const bool second = id == r1;
+#pragma unroll
+        for (int h = 0; h < G::NSPAN; ++h)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int col = frag_col(h, t, e);
+            const float add = rcv[c * D + col] * s.G[col];
+            if (second) SX(1, h, e) += add; else SX(0, h, e) += add;
+          }
+      }
+    } else {
+      const int jc = id - D;
+      if (((jc & 63) >> 4) == t && chunk_valid<D>(t)) {
+        const float gj = s.G[jc];
+        const float a0 = rcv[c * D + r0] * gj, a1 = rcv[c * D + r1] * gj;
+#pragma unroll
+        for (int h = 0; h < G::NSPAN; ++h)
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (frag_col(h, t, e) == jc) {
+              SX(0, h, e) += a0;
+              SX(1, h, e) += a1;
+            }
+      }
+    }
+  }
+}
+
+// Quantize the state held in registers (fragment layout) into the record at
+// rec (global):
+//  1. K times: the untaken line (row or column) of the largest fp64 energy of
+//     the residual (ties: lower id; rows are ids 0..D-1, columns D..2D-1) is
+//     stored as an fp32 compensator vector and zeroed; the energies of the
+//     crossing lines lose the removed squares;
+//  2. m_j from the residual's column max a_j: 1 if smoothing is off or
+//     a_j < FLT_MIN, else sqrt(a_j) or a_j;
+//  3. per row: x = (R_ij * (1/m_j)) * (127/b_i) with b_i the row max of
+//     R_ij * (1/m_j); code = round-half-even(x) clamped to [-127, 127];
+//     sigma_i = b_i / 127, or 1 with zero codes when b_i < FLT_MIN.
+// colpart / colmax: shared scratch of (D/16) x D doubles / floats.
+template <int D, class SC>
+__device__ void quantize_tile(SC &s, double *colpart, float *colmax,
+                              float2 (&S)[2][FG<D>::NSPAN][8], uint8_t *rec, const RecLayout &L,
+                              int K, int smooth) {
+  using G = FG<D>;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int r0 = 16 * warp + g, r1 = r0 + 8;
+  const bool rows_here = warp < G::NRB;
+  float *rsig = reinterpret_cast<float *>(rec + L.off_sig);
+  float *rm = reinterpret_cast<float *>(rec + L.off_m);
+  float *rcv = reinterpret_cast<float *>(rec + L.off_cv);
+  int *rcid = reinterpret_cast<int *>(rec + L.off_cid);
+
+  if (K > 0) {
+    // Thread j < D owns candidate lines j (row j) and D + j (column j): their
+    // fp64 energies and taken flags live in its registers.
+    if (rows_here) {
+      double e0 = 0.0, e1 = 0.0;
+#pragma unroll
+      for (int h = 0; h < G::NSPAN; ++h) {
+        double cp[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const double a = SX(0, h, e), b = SX(1, h, e);
+          e0 = fma(a, a, e0);
+          e1 = fma(b, b, e1);
+          cp[e] = fma(a, a, b * b);
+        }
+        butterfly_g<16>(cp, lane, AddOp());
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          if (chunk_valid<D>(t)) colpart[warp * D + frag_col(h, t, 2 * g + u)] = cp[u];
+      }
+      e0 += __shfl_xor_sync(kFull, e0, 1);
+      e0 += __shfl_xor_sync(kFull, e0, 2);
+      e1 += __shfl_xor_sync(kFull, e1, 1);
+      e1 += __shfl_xor_sync(kFull, e1, 2);
+      if (t == 0) {
+        s.rowE[r0] = e0;
+        s.rowE[r1] = e1;
+      }
+    }
+    __syncthreads();
+    double eRow = 0.0, eCol = 0.0;
+    bool tRow = false, tCol = false;
+    if (tid < D) {
+      eRow = s.rowE[tid];
+#pragma unroll
+      for (int w = 0; w < G::NRB; ++w) eCol += colpart[w * D + tid];
+    }
+    for (int c = 0; c < K; ++c) {
+      // partial argmax over this thread's two candidates, then over the warp
+      if (warp < (D + 31) / 32) {
+        double best = -1.0;
+        int bid = 0x7fffffff;
+        if (tid < D) {
+          if (!tRow) {
+            best = eRow;
+            bid = tid;
+          }
+          if (!tCol && eCol > best) {
+            best = eCol;
+            bid = D + tid;
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const double ob = __shfl_xor_sync(kFull, best, o);
+          const int oid = __shfl_xor_sync(kFull, bid, o);
+          if (ob > best || (ob == best && oid < bid)) {
+            best = ob;
+            bid = oid;
+          }
+        }
+        if (lane == 0) {
+          s.pbest[warp] = best;
+          s.pid[warp] = bid;
+        }
+      }
+      __syncthreads();
+      // every thread combines the per-warp winners (same result everywhere)
+      int id = 0x7fffffff;
+      {
+        double best = -1.0;
+#pragma unroll
+        for (int w = 0; w < (D + 31) / 32; ++w) {
+          const double e = s.pbest[w];
+          const int i2 = s.pid[w];
+          if (e > best || (e == best && i2 < id)) {
+            best = e;
+            id = i2;
+          }
+        }
+      }
+      // the owners of the line park its values in s.line and zero them
+      if (rows_here) {
+        if (id < D) {
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            if ((rr ? r1 : r0) != id || !chunk_valid<D>(t)) continue;
+#pragma unroll
+            for (int h = 0; h < G::NSPAN; ++h) {
+              float4 *dst = reinterpret_cast<float4 *>(&s.line[frag_col(h, t, 0)]);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                dst[u] = make_float4(S[rr][h][2 * u].x, S[rr][h][2 * u].y, S[rr][h][2 * u + 1].x,
+                                     S[rr][h][2 * u + 1].y);
+                S[rr][h][2 * u] = make_float2(0.0f, 0.0f);
+                S[rr][h][2 * u + 1] = make_float2(0.0f, 0.0f);
+              }
+            }
+          }
+        } else {
+          const int jc = id - D;
+          if (((jc & 63) >> 4) == t && chunk_valid<D>(t)) {
+#pragma unroll
+            for (int h = 0; h < G::NSPAN; ++h)
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                if (frag_col(h, t, e) == jc) {
+                  s.line[r0] = SX(0, h, e);
+                  s.line[r1] = SX(1, h, e);
+                  SX(0, h, e) = 0.0f;
+                  SX(1, h, e) = 0.0f;
+                }
+          }
+        }
+      }
+      __syncthreads();
+      // store the line; the crossing lines lose its squares; mark it taken
+      if (tid < D) {
+        const float v = s.line[tid];
+        rcv[c * D + tid] = v;
+        const double v2 = static_cast<double>(v) * static_cast<double>(v);
+        if (id < D) {
+          eCol -= v2;
+          if (id == tid) tRow = true;
+        } else {
+          eRow -= v2;
+          if (id == D + tid) tCol = true;
+        }
+        if (tid == 0) rcid[c] = id;
+      }
+    }
+  }
+
+  // Smoothing factors from the residual's column maxima.
+  if (rows_here) {
+#pragma unroll
+    for (int h = 0; h < G::NSPAN; ++h) {
+      float cm[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) cm[e] = fmaxf(fabsf(SX(0, h, e)), fabsf(SX(1, h, e)));
+      butterfly_g<16>(cm, lane, MaxOp());
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (chunk_valid<D>(t)) colmax[warp * D + frag_col(h, t, 2 * g + u)] = cm[u];
+    }
+  }
+  __syncthreads();
+  if (tid < D) {
+    float a = 0.0f;
+#pragma unroll
+    for (int w = 0; w < G::NRB; ++w) a = fmaxf(a, colmax[w * D + tid]);
+    float mj;
+    if (smooth == 0 || a < FLT_MIN)
+      mj = 1.0f;
+    else if (smooth == 1)
+      mj = __fsqrt_rn(a);
+    else
+      mj = a;
+    rm[tid] = mj;
+    s.invm[padc(tid)] = __frcp_rn(mj);
+  }
+  __syncthreads();
+
+  // Per-row scales and int8 codes.
+  if (rows_here) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int row = rr ? r1 : r0;
+      float bmax = 0.0f;
+#pragma unroll
+      for (int h = 0; h < G::NSPAN; ++h) {
+        if (!chunk_valid<D>(t)) continue;
+        const float4 *im4 = reinterpret_cast<const float4 *>(&s.invm[padc(frag_col(h, t, 0))]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 im = im4[u];
+          S[rr][h][2 * u] = __fmul2_rn(S[rr][h][2 * u], make_float2(im.x, im.y));
+          S[rr][h][2 * u + 1] = __fmul2_rn(S[rr][h][2 * u + 1], make_float2(im.z, im.w));
+          bmax = fmaxf(bmax, fmaxf(fmaxf(fabsf(S[rr][h][2 * u].x), fabsf(S[rr][h][2 * u].y)),
+                                   fmaxf(fabsf(S[rr][h][2 * u + 1].x),
+                                         fabsf(S[rr][h][2 * u + 1].y))));
+        }
+      }
+      bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, 1));
+      bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, 2));
+      float sg, inv;
+      if (bmax < FLT_MIN) {
+        sg = 1.0f;
+        inv = 0.0f;
+      } else {
+        sg = __fdiv_rn(bmax, 127.0f);
+        inv = __fdiv_rn(127.0f, bmax);
+      }
+      if (t == 0) rsig[row] = sg;
+      const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+      for (int h = 0; h < G::NSPAN; ++h) {
+        if (!chunk_valid<D>(t)) continue;
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          // |x| <= 127 (1 + 2^-23) by construction; the clamp guards the bound
+          const float2 xa = __fmul2_rn(S[rr][h][2 * u], inv2);
+          const float2 xb = __fmul2_rn(S[rr][h][2 * u + 1], inv2);
+          const float x0 = fminf(fmaxf(xa.x, -127.0f), 127.0f) + kRoundMagic;
+          const float x1 = fminf(fmaxf(xa.y, -127.0f), 127.0f) + kRoundMagic;
+          const float x2 = fminf(fmaxf(xb.x, -127.0f), 127.0f) + kRoundMagic;
+          const float x3 = fminf(fmaxf(xb.y, -127.0f), 127.0f) + kRoundMagic;
+          w[u] = __byte_perm(__byte_perm(__float_as_uint(x0), __float_as_uint(x1), 0x0040u),
+                             __byte_perm(__float_as_uint(x2), __float_as_uint(x3), 0x0040u),
+                             0x5410u);
+        }
+        *reinterpret_cast<uint4 *>(rec + static_cast<size_t>(row) * D + frag_col(h, t, 0)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Decode step
+// ---------------------------------------------------------------------------
+
+// Bulk copy of a tile's record into a ring slot (one thread); the mbarrier
+// is told to expect its bytes but not arrived on.
+template <int D, bool BF16, bool KDA>
+__device__ __forceinline__ void issue_record(const KParams &p, uint8_t *slot,
+                                             unsigned long long *bar, int tile) {
+  const uint32_t rec_b = static_cast<uint32_t>(p.L.bytes);
+  mbar_expect_tx(bar, rec_b);
+  bulk_g2s(slot, p.records + static_cast<size_t>(tile) * rec_b, rec_b, bar);
+}
+
+// Bulk copies of the rest of a tile (buffered tokens, inputs) into its ring
+// slot, then the arrival that lets the slot's phase complete once every byte
+// has landed (one thread).  n < 0: nothing more to copy (skipped tile).
+template <int D, bool BF16, bool KDA>
+__device__ __forceinline__ void issue_rest(const KParams &p, uint8_t *slot,
+                                           unsigned long long *bar, int tile, int n, int coord) {
+  using L = SL<D, BF16, KDA>;
+  const L lay(p.L.bytes);
+  if (n < 0) {
+    mbar_arrive_expect_tx(bar, 0);
+    return;
+  }
+  const int b = coord >> 12, hk = (coord >> 1) & 2047;
+  const uint32_t bd_b = static_cast<uint32_t>(n) * D * 4;
+  const uint32_t bk_b = static_cast<uint32_t>(n) * D * L::IB;
+  const uint32_t bg_b = KDA ? bd_b : kGdnGateStride * 4;
+  const uint32_t in_b = D * L::IB;
+  const uint32_t total = bd_b + bk_b + bg_b + 3 * in_b + (KDA ? static_cast<uint32_t>(D) * 4 : 0u);
+  mbar_arrive_expect_tx(bar, total);
+  if (n > 0) {
+    bulk_g2s(slot + lay.bd, p.buf_d + static_cast<size_t>(tile) * p.W * D, bd_b, bar);
+    bulk_g2s(slot + lay.bk,
+             static_cast<const uint8_t *>(p.buf_k) +
+                 (static_cast<size_t>(b) * p.Hk + hk) * p.W * D * L::IB,
+             bk_b, bar);
+    if (KDA) bulk_g2s(slot + lay.bg, p.buf_g + static_cast<size_t>(tile) * p.W * D, bg_b, bar);
+  }
+  if (!KDA) bulk_g2s(slot + lay.bg, p.buf_g + static_cast<size_t>(tile) * kGdnGateStride,
+                     bg_b, bar);
+  const size_t qk = (static_cast<size_t>(b) * p.Hk + hk) * D * L::IB;
+  bulk_g2s(slot + lay.q, static_cast<const uint8_t *>(p.q) + qk, in_b, bar);
+  bulk_g2s(slot + lay.k, static_cast<const uint8_t *>(p.k) + qk, in_b, bar);
+  bulk_g2s(slot + lay.v, static_cast<const uint8_t *>(p.v) + static_cast<size_t>(tile) * in_b,
+           in_b, bar);
+  if (KDA) bulk_g2s(slot + lay.a, p.alpha + static_cast<size_t>(tile) * D, D * 4, bar);
+}
+
+// GDN with bf16 inputs: the buffer coefficients of all slots from one warp.
+// Raw dots k_s . k_t and k_s . q_t for slots s = 0..15 run on the bf16 tensor
+// path (keys and queries are bf16, so every product is exact; fp32
+// accumulation); slot n is the current key itself.  The scalar decay ratios
+// rho_s = prod_{s < s' <= n} alpha_{s'} come from a suffix-product scan over
+// the lanes (lane s holds alpha_s).  Writes c_s = rho_s (k_s . k_t) and
+// a_s = rho_s (k_s . q_t) for s < n, a_n = k_t . q_t, and rho_s for s <= n.
+template <int D, class SC>
+__device__ __forceinline__ void coef_mma(SC &s, const __nv_bfloat16 *sbk,
+                                         const __nv_bfloat16 *sk, const __nv_bfloat16 *sq,
+                                         const float *sbg, float alpha0, int n) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  const __nv_bfloat16 *row0 = (g < n) ? sbk + g * D : (g == n ? sk : nullptr);
+  const __nv_bfloat16 *row1 = (g + 8 < n) ? sbk + (g + 8) * D : (g + 8 == n ? sk : nullptr);
+  const __nv_bfloat16 *vec = (g == 0) ? sk : (g == 1 ? sq : nullptr);
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int ch = 0; ch < D / 32; ++ch) {
+    const int off = 32 * ch + 8 * t;
+    const uint4 a0 = row0 ? *reinterpret_cast<const uint4 *>(row0 + off) : zero;
+    const uint4 a1 = row1 ? *reinterpret_cast<const uint4 *>(row1 + off) : zero;
+    const uint4 bb = vec ? *reinterpret_cast<const uint4 *>(vec + off) : zero;
+    mma_bf16(c, a0.x, a1.x, a0.y, a1.y, bb.x, bb.y);
+    mma_bf16(c, a0.z, a1.z, a0.w, a1.w, bb.z, bb.w);
+  }
+  float P = (lane < n) ? sbg[lane] : (lane == n ? alpha0 : 1.0f);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float v = __shfl_down_sync(kFull, P, o);
+    if (lane + o < 32) P *= v;
+  }
+  // lane s now holds prod_{s' >= s} alpha_{s'}; rho_s is lane s+1's value
+  const float rho0 = __shfl_sync(kFull, P, (g + 1) & 31);
+  const float rho1 = __shfl_sync(kFull, P, (g + 9) & 31);
+  if (t == 0) {
+    if (g <= n) {
+      s.cc[g] = rho0 * c[0];
+      s.aa[g] = rho0 * c[1];
+      s.rho[g] = rho0;
+    }
+    if (g + 8 <= n) {
+      s.cc[g + 8] = rho1 * c[2];
+      s.aa[g + 8] = rho1 * c[3];
+      s.rho[g + 8] = rho1;
+    }
+  }
+}
+
+// Four radix-128 int8 digits of u (|u| < 64), packed into the bytes of d.
+__device__ __forceinline__ void digits4(float u, uint32_t (&d)[4], int shift) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float biased = u + kRoundMagic;
+    d[i] |= (__float_as_uint(biased) & 0xffu) << shift;
+    u = (u - (biased - kRoundMagic)) * 128.0f;
+  }
+}
+
+// Power-of-two factor 2^(6-E) with max|x| = M < 2^E (M > 0), and its inverse
+// 2^(E-6); exact.  Tiny M takes the library path.
+__device__ __forceinline__ void digit_scales(float M, float &up, float &down) {
+  const int eb = static_cast<int>((__float_as_uint(M) >> 23) & 0xffu);
+  if (eb >= 6) {
+    up = __uint_as_float(static_cast<uint32_t>(259 - eb) << 23);
+    down = digit_scale(M);
+  } else {
+    int E;
+    frexpf(M, &E);
+    up = ldexpf(1.0f, 6 - E);
+    down = ldexpf(1.0f, E - 6);
+  }
+}
+
+// GDN with bf16 inputs: all per-channel work of a tile in one warp; lane l
+// takes the CPL = D/32 consecutive channels CPL*l ... CPL*l + CPL-1.  Writes
+// q, k, v (fp32), Gamma, m o Gamma, the digits of x_q and x_k with their
+// scales, the row-compensator partial dots (cpart[c][0]), and appends k_t.
+template <int D, class SC>
+__device__ __forceinline__ void channel_warp_fast(const KParams &p, SC &s,
+                                                  const __nv_bfloat16 *sq,
+                                                  const __nv_bfloat16 *sk,
+                                                  const __nv_bfloat16 *sv, const float *sbg,
+                                                  const float *rm, const float *rcv,
+                                                  const int *rcid, float alpha0, int n,
+                                                  size_t key_slot, bool writes_key) {
+  constexpr int CPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int j0 = CPL * lane;
+  // window gate Gamma_t = prod of the n buffered gates and the current one
+  float P = (lane < n) ? sbg[lane] : (lane == n ? alpha0 : 1.0f);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) P *= __shfl_xor_sync(kFull, P, o);
+  const float Gm = P;
+  float q[CPL], k[CPL], xq[CPL], xk[CPL];
+  float mq = 0.0f, mk = 0.0f;
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    const int j = j0 + c;
+    q[c] = __bfloat162float(sq[j]);
+    k[c] = __bfloat162float(sk[j]);
+    const float mj = rm[j];
+    s.qf[j] = q[c];
+    s.kf[j] = k[c];
+    s.vf[j] = __bfloat162float(sv[j]);
+    s.G[j] = Gm;
+    s.mG[padc(j)] = mj * Gm;
+    xq[c] = mj * (Gm * q[c]);
+    xk[c] = mj * (Gm * k[c]);
+    mq = fmaxf(mq, fabsf(xq[c]));
+    mk = fmaxf(mk, fabsf(xk[c]));
+  }
+  if (writes_key) {
+    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.buf_k) + key_slot;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) dst[j0 + c] = sk[j0 + c];
+  }
+  mq = warp_max_abs(mq);
+  mk = warp_max_abs(mk);
+  float upq = 0.0f, dnq = 0.0f, upk = 0.0f, dnk = 0.0f;
+  if (mq > 0.0f) digit_scales(mq, upq, dnq);
+  if (mk > 0.0f) digit_scales(mk, upk, dnk);
+  uint32_t dq[4] = {0u, 0u, 0u, 0u}, dk[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    digits4(xq[c] * upq, dq, 8 * c);
+    digits4(xk[c] * upk, dk, 8 * c);
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    if constexpr (CPL == 4) {
+      *reinterpret_cast<uint32_t *>(&s.dig[r][j0]) = dq[r];
+      *reinterpret_cast<uint32_t *>(&s.dig[4 + r][j0]) = dk[r];
+    } else {
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        s.dig[r][j0 + c] = static_cast<int8_t>((dq[r] >> (8 * c)) & 0xffu);
+        s.dig[4 + r][j0 + c] = static_cast<int8_t>((dk[r] >> (8 * c)) & 0xffu);
+      }
+    }
+  }
+  if (lane == 0) {
+    s.xscale[0] = dnq;
+    s.xscale[1] = dnk;
+  }
+  // row-compensator lines dotted with Gamma o q and Gamma o k
+  for (int c0 = 0; c0 < p.K; c0 += 4) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = c0 + i;
+      float aq = 0.0f, ak = 0.0f;
+      if (c < p.K && rcid[c] < D) {
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) {
+          const float cvj = rcv[c * D + j0 + u];
+          aq = fmaf(cvj, q[u], aq);
+          ak = fmaf(cvj, k[u], ak);
+        }
+      }
+      v[2 * i] = Gm * aq;
+      v[2 * i + 1] = Gm * ak;
+    }
+    const float tot = warp_sum8(v, lane);
+    const int vi = (lane >> 2) & 7, c = c0 + (vi >> 1);
+    if ((lane & 3) == 0 && c < p.K) s.cpart[c][0][vi & 1] = tot;
+  }
+}
+
+// One token for one staged tile: outputs, buffer append, and on the W-th token
+// the fold and requantization.  Three phases separated by CTA barriers:
+//  A  channel threads (one per key channel j): inputs, decay ratios applied to
+//     the buffered keys, Gamma, x = m o Gamma o {q, k} and its per-warp max;
+//     appends k_t and the KDA gate.  The other warps fetch their code
+//     fragments.
+//  B  channel threads: the int8 digits of x_q, x_k and the row-compensator
+//     dots; the other warps: the buffer coefficients c_s, a_s.
+//  C  every row warp: y_q, y_k for its 16 rows on the int8 tensor path, then
+//     finishes its rows (buffer sums split over the 4 lanes of a row):
+//     d_t = beta (v - y_k - sum c_s d_s), o_t = y_q + sum a_s d_s + a_t d_t.
+template <int D, bool BF16, bool KDA, class SC>
+__device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *slot,
+                                             int tile, int n, int coord, float alpha0,
+                                             float beta) {
+  using G = FG<D>;
+  using L = SL<D, BF16, KDA>;
+  using IT = in_t<BF16>;
+  constexpr int CW = (D + 31) / 32;  // channel warps
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int b = coord >> 12, hk = (coord >> 1) & 2047;
+  const bool writes_key = (coord & 1) != 0;
+  const uint8_t *codes = slot;
+  const float *rsig = reinterpret_cast<const float *>(slot + p.L.off_sig);
+  const float *rm = reinterpret_cast<const float *>(slot + p.L.off_m);
+  const float *rcv = reinterpret_cast<const float *>(slot + p.L.off_cv);
+  const int *rcid = reinterpret_cast<const int *>(slot + p.L.off_cid);
+  const L lay(p.L.bytes);
+  float *sbd = reinterpret_cast<float *>(slot + lay.bd);
+  const IT *sbk = reinterpret_cast<const IT *>(slot + lay.bk);
+  const float *sbg = reinterpret_cast<const float *>(slot + lay.bg);
+  const IT *sq = reinterpret_cast<const IT *>(slot + lay.q);
+  const IT *sk = reinterpret_cast<const IT *>(slot + lay.k);
+  const IT *sv = reinterpret_cast<const IT *>(slot + lay.v);
+  const float *sa = reinterpret_cast<const float *>(slot + lay.a);
+
+  // ---- Phases A and B ----
+  constexpr bool kFast = DecodeTraits<D, BF16, KDA>::kFast;
+  constexpr int CWP = kFast ? 1 : CW;  // warps holding compensator partial dots
+  uint4 A[2][G::NSPAN];
+  if constexpr (kFast) {
+    // one warp for the channels, one for the buffer coefficients; the other
+    // row warps fetch their code fragments
+    if (warp == 0) {
+      channel_warp_fast<D>(p, s, reinterpret_cast<const __nv_bfloat16 *>(sq),
+                           reinterpret_cast<const __nv_bfloat16 *>(sk),
+                           reinterpret_cast<const __nv_bfloat16 *>(sv), sbg, rm, rcv, rcid,
+                           alpha0, n,
+                           ((static_cast<size_t>(b) * p.Hk + hk) * p.W + n) * D, writes_key);
+      if (lane == 0) p.buf_g[static_cast<size_t>(tile) * kGdnGateStride + n] = alpha0;
+    } else if (warp == 1) {
+      coef_mma<D>(s, reinterpret_cast<const __nv_bfloat16 *>(sbk),
+                  reinterpret_cast<const __nv_bfloat16 *>(sk),
+                  reinterpret_cast<const __nv_bfloat16 *>(sq), sbg, alpha0, n);
+    } else if (warp < G::NRB) {
+      load_codes<D>(codes, A);
+    }
+    __syncthreads();
+  } else {
+    // ---- Phase A ----
+  float xq = 0.0f, xk = 0.0f;
+  if (tid < D) {
+    const int j = tid;
+    const float qj = to_f(sq[j]), kj = to_f(sk[j]);
+    s.qf[j] = qj;
+    s.kf[j] = kj;
+    s.vf[j] = to_f(sv[j]);
+    float acc;
+    if constexpr (kFast) {
+      // window gate Gamma_t = prod of the n buffered gates and the current one
+      float P = (lane < n) ? sbg[lane] : (lane == n ? alpha0 : 1.0f);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) P *= __shfl_xor_sync(kFull, P, o);
+      acc = P;
+    } else {
+      // decay ratios prod_{s < s' <= t} alpha_{s'} as running products from
+      // the current token backwards, applied to the buffered keys
+      acc = KDA ? sa[j] : alpha0;
+      for (int sl = n - 1; sl >= 0; --sl) {
+        s.kt[sl][padc(j)] = to_f(sbk[sl * D + j]) * acc;
+        acc *= KDA ? sbg[sl * D + j] : sbg[sl];
+      }
+      s.kt[n][padc(j)] = kj;
+    }
+    s.G[j] = acc;
+    const float mj = rm[j];
+    xq = mj * (acc * qj);
+    xk = mj * (acc * kj);
+    s.mG[padc(j)] = mj * acc;
+    if (writes_key)
+      reinterpret_cast<IT *>(p.buf_k)[((static_cast<size_t>(b) * p.Hk + hk) * p.W + n) * D + j] =
+          sk[j];
+    if constexpr (KDA) p.buf_g[(static_cast<size_t>(tile) * p.W + n) * D + j] = sa[j];
+    const float mq = warp_max_abs(xq), mk = warp_max_abs(xk);
+    if (lane == 0) {
+      s.xmax[0][warp] = mq;
+      s.xmax[1][warp] = mk;
+    }
+    // row-compensator lines dotted with Gamma o q and Gamma o k: per-warp
+    // partials, four lines per transposed reduction
+    const float gq = acc * qj, gk = acc * kj;
+    for (int c0 = 0; c0 < p.K; c0 += 4) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = c0 + i;
+        const float cvj = (c < p.K && rcid[c] < D) ? rcv[c * D + j] : 0.0f;
+        v[2 * i] = cvj * gq;
+        v[2 * i + 1] = cvj * gk;
+      }
+      const float tot = warp_sum8(v, lane);
+      const int vi = (lane >> 2) & 7, c = c0 + (vi >> 1);
+      if ((lane & 3) == 0 && c < p.K) s.cpart[c][warp][vi & 1] = tot;
+    }
+  } else if (warp < G::NRB) {
+    load_codes<D>(codes, A);
+  }
+  if constexpr (kFast) {
+    if (warp == CW) coef_mma<D>(s, reinterpret_cast<const __nv_bfloat16 *>(sbk),
+                                reinterpret_cast<const __nv_bfloat16 *>(sk),
+                                reinterpret_cast<const __nv_bfloat16 *>(sq), sbg, alpha0, n);
+  }
+  if constexpr (!KDA) {
+    if (tid == 0) p.buf_g[static_cast<size_t>(tile) * kGdnGateStride + n] = alpha0;
+  }
+  __syncthreads();
+
+  // ---- Phase B ----
+  if (tid < D) {
+    float Mq = 0.0f, Mk = 0.0f;
+#pragma unroll
+    for (int w = 0; w < CW; ++w) {
+      Mq = fmaxf(Mq, s.xmax[0][w]);
+      Mk = fmaxf(Mk, s.xmax[1][w]);
+    }
+    split_digits(xq, Mq, &s.dig[0][tid], G::DIGW);
+    split_digits(xk, Mk, &s.dig[4][tid], G::DIGW);
+    if (tid == 0) {
+      s.xscale[0] = digit_scale(Mq);
+      s.xscale[1] = digit_scale(Mk);
+    }
+  } else if constexpr (!kFast) {
+    // c_s = kt_s . k and a_s = kt_s . q for the buffered tokens; a_t = k . q
+    for (int sl = warp - CW; sl <= n; sl += kWarps - CW) {
+      float c = 0.0f, a = 0.0f;
+      for (int j = lane; j < D; j += 32) {
+        const float kv = s.kt[sl][padc(j)];
+        c = fmaf(kv, s.kf[j], c);
+        a = fmaf(kv, s.qf[j], a);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        c += __shfl_xor_sync(kFull, c, o);
+        a += __shfl_xor_sync(kFull, a, o);
+      }
+      if (lane == 0) {
+        s.cc[sl] = c;
+        s.aa[sl] = a;
+      }
+    }
+  }
+  __syncthreads();
+
+  }
+
+  // ---- Phase C ----
+  if (warp < G::NRB) {
+    if (kFast ? warp < 2 : tid < D) load_codes<D>(codes, A);
+    int acc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int hh = 0; hh < G::NSPAN; ++hh) {
+      uint4 Bw = make_uint4(0, 0, 0, 0);
+      if (chunk_valid<D>(t))
+        Bw = *reinterpret_cast<const uint4 *>(&s.dig[g][frag_col(hh, t, 0)]);
+      mma_s8(acc, A[0][hh].x, A[1][hh].x, A[0][hh].y, A[1][hh].y, Bw.x, Bw.y);
+      mma_s8(acc, A[0][hh].z, A[1][hh].z, A[0][hh].w, A[1][hh].w, Bw.z, Bw.w);
+    }
+    // lane (g, t) holds digits 2t, 2t+1 of rows r0 (acc 0,1) and r0+8 (acc 2,3);
+    // t = 0,1: x_q digits 0-1, 2-3; t = 2,3: x_k digits 0-1, 2-3.
+    float p0 = static_cast<float>(acc[0]) + static_cast<float>(acc[1]) * (1.0f / 128.0f);
+    float p1 = static_cast<float>(acc[2]) + static_cast<float>(acc[3]) * (1.0f / 128.0f);
+    if (t & 1) {
+      p0 *= 1.0f / 16384.0f;
+      p1 *= 1.0f / 16384.0f;
+    }
+    p0 += __shfl_xor_sync(kFull, p0, 1);
+    p1 += __shfl_xor_sync(kFull, p1, 1);
+    const int r0 = 16 * warp + g, r1 = r0 + 8;
+    const int base_lane = lane & ~3;
+    const float sq0 = s.xscale[0], sk0 = s.xscale[1];
+    float yq0 = __shfl_sync(kFull, p0, base_lane) * sq0 * rsig[r0];
+    float yq1 = __shfl_sync(kFull, p1, base_lane) * sq0 * rsig[r1];
+    float yk0 = __shfl_sync(kFull, p0, base_lane | 2) * sk0 * rsig[r0];
+    float yk1 = __shfl_sync(kFull, p1, base_lane | 2) * sk0 * rsig[r1];
+    // buffer sums and compensator lines, split over the 4 lanes of the rows:
+    // xa collects what adds to o, xc what is subtracted from v
+    float xc0 = 0.0f, xa0 = 0.0f, xc1 = 0.0f, xa1 = 0.0f;
+    for (int sl = t; sl < n; sl += 4) {
+      const float c = s.cc[sl], a = s.aa[sl];
+      const float d0 = sbd[sl * D + r0], d1 = sbd[sl * D + r1];
+      xc0 = fmaf(c, d0, xc0);
+      xa0 = fmaf(a, d0, xa0);
+      xc1 = fmaf(c, d1, xc1);
+      xa1 = fmaf(a, d1, xa1);
+    }
+    for (int c = t; c < p.K; c += 4) {
+      const int id = rcid[c];
+      if (id < D) {
+        if (id == r0 || id == r1) {
+          float dq = 0.0f, dk = 0.0f;
+#pragma unroll
+          for (int w = 0; w < CWP; ++w) {
+            dq += s.cpart[c][w][0];
+            dk += s.cpart[c][w][1];
+          }
+          if (id == r0) {
+            xa0 += dq;
+            xc0 += dk;
+          } else {
+            xa1 += dq;
+            xc1 += dk;
+          }
+        }
+      } else {
+        const int jc = id - D;
+        const float gj = s.G[jc];
+        const float gq = gj * s.qf[jc], gk = gj * s.kf[jc];
+        const float c0 = rcv[c * D + r0], c1 = rcv[c * D + r1];
+        xa0 = fmaf(c0, gq, xa0);
+        xc0 = fmaf(c0, gk, xc0);
+        xa1 = fmaf(c1, gq, xa1);
+        xc1 = fmaf(c1, gk, xc1);
+      }
+    }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      xc0 += __shfl_xor_sync(kFull, xc0, o);
+      xa0 += __shfl_xor_sync(kFull, xa0, o);
+      xc1 += __shfl_xor_sync(kFull, xc1, o);
+      xa1 += __shfl_xor_sync(kFull, xa1, o);
+    }
+    if (t < 2) {
+      const int row = t ? r1 : r0;
+      const float yq = t ? yq1 : yq0, yk = t ? yk1 : yk0;
+      const float xc = t ? xc1 : xc0, xa = t ? xa1 : xa0;
+      const float dt = beta * (s.vf[row] - yk - xc);
+      const float o = fmaf(s.aa[n], dt, yq + xa);
+      st_out(p.out, static_cast<size_t>(tile) * D + row, o, p.out_bf16);
+      p.buf_d[(static_cast<size_t>(tile) * p.W + n) * D + row] = dt;
+      sbd[n * D + row] = dt;
+    }
+  }
+  if (n + 1 < p.W) {
+    if (tid == 0) p.buf_n[tile] = n + 1;
+    return;
+  }
+
+  // Window boundary: fold the W buffered tokens and requantize.
+  __syncthreads();
+  float2 S[2][G::NSPAN][8];
+  uint4 Af[2][G::NSPAN];
+  if (warp < G::NRB) load_codes<D>(codes, Af);
+  const float *kt;
+  if constexpr (DecodeTraits<D, BF16, KDA>::kFast) {
+    // scaled keys from the staged keys and the scalar ratios; at d = 128 they
+    // go over the staged codes, which are now in registers
+    float *ktw;
+    if constexpr (DecodeTraits<D, BF16, KDA>::kKtOverCodes) {
+      __syncthreads();
+      ktw = reinterpret_cast<float *>(slot);
+    } else {
+      ktw = &s.kt[0][0];
+    }
+    if (tid < D) {
+      for (int sl = 0; sl < n; ++sl)
+        ktw[sl * G::PADW + padc(tid)] = to_f(sbk[sl * D + tid]) * s.rho[sl];
+      ktw[n * G::PADW + padc(tid)] = s.kf[tid];
+    }
+    __syncthreads();
+    kt = ktw;
+  } else {
+    kt = &s.kt[0][0];
+  }
+  if (warp < G::NRB) build_state<D>(s, kt, Af, rsig, rcv, rcid, sbd, n + 1, p.K, S);
+  __syncthreads();  // the staged codes and keys are now free for the quantizer's scratch
+  quantize_tile<D>(s, reinterpret_cast<double *>(slot + L::QS_COLPART),
+                   reinterpret_cast<float *>(slot + L::QS_COLMAX), S,
+                   p.records + static_cast<size_t>(tile) * p.L.bytes, p.L, p.K, p.smooth);
+  if (tid == 0) p.buf_n[tile] = 0;
+}
+
+template <int D, bool BF16, bool KDA>
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
+  using L = SL<D, BF16, KDA>;
+  using TR = DecodeTraits<D, BF16, KDA>;
+  constexpr int kStages = TR::kStages;
+  using SC = Scratch<D, !TR::kKtOverCodes>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int slot_bytes = L(p.L.bytes).bytes;
+  SC &s = *reinterpret_cast<SC *>(smem + kStages * slot_bytes);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tiles = p.B * p.Hv;
+
+  // This CTA's tiles are blockIdx.x + i * gridDim.x.  Without a mask every
+  // tile keeps its position in the list, so the first slots' record copies go
+  // out before the phases are known; with a mask the list is compacted to the
+  // active sequences first.
+  const int mine = (tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                   static_cast<int>(gridDim.x);
+  const bool speculate = p.mask == nullptr;
+  if (tid == 0) {
+    s.abort = 0;
+    for (int st = 0; st < kStages; ++st) mbar_init(&s.bar[st], 1);
+    fence_mbar_init();
+    if (speculate)
+      for (int st = 0; st < kStages && st < mine; ++st)
+        issue_record<D, BF16, KDA>(p, smem + st * slot_bytes, &s.bar[st],
+                                   blockIdx.x + st * gridDim.x);
+  }
+  int keep = 0, tile = 0, n = -1, coord = 0;
+  float a0 = 0.0f, b0 = 0.0f;
+  if (tid < mine) {
+    tile = blockIdx.x + tid * gridDim.x;
+    const int b = tile / p.Hv, h = tile - b * p.Hv, group = p.Hv / p.Hk;
+    coord = (b << 12) | ((h / group) << 1) | ((h % group == 0) ? 1 : 0);
+    if (speculate || p.mask[b] != 0) {
+      keep = 1;
+      n = p.buf_n[tile];
+      if (n >= 0 && n < p.W) {
+        if (!KDA) a0 = p.alpha[tile];
+        b0 = p.beta[tile];
+      } else {
+        atomicOr(p.err, kErrBadPhase);
+        n = -1;
+      }
+    }
+  }
+  const unsigned ball = __ballot_sync(kFull, keep);
+  if (lane == 0) s.warp_cnt[warp] = __popc(ball);
+  __syncthreads();
+  int base = 0, count = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    base += (w < warp) ? s.warp_cnt[w] : 0;
+    count += s.warp_cnt[w];
+  }
+  if (keep) {
+    const int pos = base + __popc(ball & ((1u << lane) - 1u));
+    s.tl_tile[pos] = tile;
+    s.tl_n[pos] = n;
+    s.tl_coord[pos] = coord;
+    s.tl_a[pos] = a0;
+    s.tl_b[pos] = b0;
+  }
+  __syncthreads();
+
+  if (tid == 0)
+    for (int st = 0; st < kStages && st < count; ++st) {
+      uint8_t *slot = smem + st * slot_bytes;
+      if (!speculate) issue_record<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[st]);
+      issue_rest<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[st], s.tl_n[st], s.tl_coord[st]);
+    }
+
+  int i = 0;
+  for (; i < count; ++i) {
+    const int st = i % kStages;
+    const uint32_t parity = static_cast<uint32_t>(i / kStages) & 1u;
+    if (!mbar_wait_bounded(&s.bar[st], parity)) s.abort = 1;
+    __syncthreads();
+    if (s.abort) break;
+    if (s.tl_n[i] >= 0)
+      process_tile<D, BF16, KDA>(p, s, smem + st * slot_bytes, s.tl_tile[i], s.tl_n[i],
+                                 s.tl_coord[i], s.tl_a[i], s.tl_b[i]);
+    // The slot was read and written through the generic proxy; order that
+    // before the bulk copy that refills it.
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0 && i + kStages < count) {
+      const int nx = i + kStages;
+      uint8_t *slot = smem + st * slot_bytes;
+      issue_record<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[nx]);
+      issue_rest<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[nx], s.tl_n[nx], s.tl_coord[nx]);
+    }
+  }
+  if (i < count) {
+    // A copy did not complete in time: flag it, then give the copies still in
+    // flight into this CTA's shared memory a bounded chance to land.
+    if (tid == 0) {
+      atomicOr(p.err, kErrTimeout);
+      const int last = (i + kStages < count) ? i + kStages : count;
+      for (int k = i; k < last; ++k)
+        mbar_wait_bounded(&s.bar[k % kStages], static_cast<uint32_t>(k / kStages) & 1u);
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Flush (fold a partial window), dequantize, init
+// ---------------------------------------------------------------------------
+
+// Loads a tile's record and n buffered tokens into a slot with plain 16-byte
+// loads (the whole CTA).
+template <int D, bool BF16, bool KDA>
+__device__ __forceinline__ void load_slot(const KParams &p, uint8_t *slot, int tile, int n) {
+  using L = SL<D, BF16, KDA>;
+  const L lay(p.L.bytes);
+  const int b = tile / p.Hv, h = tile - b * p.Hv, hk = h / (p.Hv / p.Hk);
+  auto copy = [&](uint8_t *dst, const void *src, int bytes) {
+    const uint4 *s4 = static_cast<const uint4 *>(src);
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+    for (int k = threadIdx.x; k < bytes / 16; k += kThreads) d4[k] = s4[k];
+  };
+  copy(slot, p.records + static_cast<size_t>(tile) * p.L.bytes, p.L.bytes);
+  if (n > 0) {
+    copy(slot + lay.bd, p.buf_d + static_cast<size_t>(tile) * p.W * D, n * D * 4);
+    copy(slot + lay.bk,
+         static_cast<const uint8_t *>(p.buf_k) + (static_cast<size_t>(b) * p.Hk + hk) * p.W * D * L::IB,
+         n * D * L::IB);
+    if (KDA) copy(slot + lay.bg, p.buf_g + static_cast<size_t>(tile) * p.W * D, n * D * 4);
+  }
+  if (!KDA) copy(slot + lay.bg, p.buf_g + static_cast<size_t>(tile) * kGdnGateStride,
+                 kGdnGateStride * 4);
+}
+
+// MODE 0: flush selected tiles with 0 < n < W.  MODE 1: write the fp32 state
+// (the window base, or the current state with include_buffer).
+template <int D, bool BF16, bool KDA, int MODE>
+__global__ void __launch_bounds__(kThreads) fold_kernel(const KParams p) {
+  using G = FG<D>;
+  using L = SL<D, BF16, KDA>;
+  using IT = in_t<BF16>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t *slot = smem;
+  const L lay(p.L.bytes);
+  Scratch<D, true> &s = *reinterpret_cast<Scratch<D, true> *>(smem + lay.bytes);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int tile = blockIdx.x;
+  const int b = tile / p.Hv;
+  if (MODE == 0 && p.mask != nullptr && p.mask[b] == 0) return;
+  int n = p.buf_n[tile];
+  if (n < 0 || n >= p.W) {
+    if (tid == 0) atomicOr(p.err, kErrBadPhase);
+    return;
+  }
+  if (MODE == 0 && n == 0) return;
+  if (MODE == 1 && !p.include_buffer) n = 0;
+  load_slot<D, BF16, KDA>(p, slot, tile, n);
+  __syncthreads();
+  const float *rsig = reinterpret_cast<const float *>(slot + p.L.off_sig);
+  const float *rm = reinterpret_cast<const float *>(slot + p.L.off_m);
+  const float *rcv = reinterpret_cast<const float *>(slot + p.L.off_cv);
+  const int *rcid = reinterpret_cast<const int *>(slot + p.L.off_cid);
+  const float *sbd = reinterpret_cast<const float *>(slot + lay.bd);
+  const IT *sbk = reinterpret_cast<const IT *>(slot + lay.bk);
+  const float *sbg = reinterpret_cast<const float *>(slot + lay.bg);
+  if (tid < D) {
+    const int j = tid;
+    float acc = 1.0f;
+    for (int sl = n - 1; sl >= 0; --sl) {
+      s.kt[sl][padc(j)] = to_f(sbk[sl * D + j]) * acc;
+      acc *= KDA ? sbg[sl * D + j] : sbg[sl];
+    }
+    s.G[j] = acc;
+    s.mG[padc(j)] = rm[j] * acc;
+  }
+  __syncthreads();
+  float2 S[2][G::NSPAN][8];
+  if (warp < G::NRB) {
+    uint4 A[2][G::NSPAN];
+    load_codes<D>(slot, A);
+    build_state<D>(s, &s.kt[0][0], A, rsig, rcv, rcid, sbd, n, p.K, S);
+  }
+  if constexpr (MODE == 0) {
+    __syncthreads();
+    quantize_tile<D>(s, reinterpret_cast<double *>(slot + L::QS_COLPART),
+                     reinterpret_cast<float *>(slot + L::QS_COLMAX), S,
+                     p.records + static_cast<size_t>(tile) * p.L.bytes, p.L, p.K, p.smooth);
+    if (tid == 0) p.buf_n[tile] = 0;
+  } else if (warp < G::NRB) {
+    float *dst = p.S_out + static_cast<size_t>(tile) * D * D;
+    const int r0 = 16 * warp + g;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+      for (int hh = 0; hh < G::NSPAN; ++hh) {
+        if (!chunk_valid<D>(t)) continue;
+        float4 *row = reinterpret_cast<float4 *>(dst + static_cast<size_t>(r0 + 8 * rr) * D +
+                                                 frag_col(hh, t, 0));
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          row[u] = make_float4(S[rr][hh][2 * u].x, S[rr][hh][2 * u].y, S[rr][hh][2 * u + 1].x,
+                               S[rr][hh][2 * u + 1].y);
+      }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) init_kernel(const KParams p) {
+  using G = FG<D>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t *qscr = smem;  // D*D bytes of quantizer scratch
+  Scratch<D, false> &s = *reinterpret_cast<Scratch<D, false> *>(smem + D * D);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int tile = blockIdx.x;
+  const int b = tile / p.Hv;
+  if (p.mask != nullptr && p.mask[b] == 0) return;
+  float2 S[2][G::NSPAN][8];
+  if (warp < G::NRB) {
+    const float *src = p.S_in + static_cast<size_t>(tile) * D * D;
+    const int r0 = 16 * warp + g;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+      for (int hh = 0; hh < G::NSPAN; ++hh) {
+        if (!chunk_valid<D>(t)) {
+#pragma unroll
+          for (int e2 = 0; e2 < 8; ++e2) S[rr][hh][e2] = make_float2(0.0f, 0.0f);
+          continue;
+        }
+        const float4 *row = reinterpret_cast<const float4 *>(
+            src + static_cast<size_t>(r0 + 8 * rr) * D + frag_col(hh, t, 0));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 v = __ldcs(row + u);
+          S[rr][hh][2 * u] = make_float2(v.x, v.y);
+          S[rr][hh][2 * u + 1] = make_float2(v.z, v.w);
+        }
+      }
+  }
+  quantize_tile<D>(s, reinterpret_cast<double *>(qscr),
+                   reinterpret_cast<float *>(qscr + G::NRB * D * 8), S,
+                   p.records + static_cast<size_t>(tile) * p.L.bytes, p.L, p.K, p.smooth);
+  if (tid == 0) p.buf_n[tile] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// Launch plumbing
+// ---------------------------------------------------------------------------
+
+// Per-device, per-kernel, per-K launch facts, computed once.
+struct LaunchInfo {
+  int ready;
+  int sms;
+  int ctas_per_sm;
+};
+
+template <typename Kern>
+cudaError_t prepare(Kern kernel, size_t smem, size_t smem_max, int K,
+                    LaunchInfo (&cache)[32][kMaxComp + 1], LaunchInfo &out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  LaunchInfo &li = cache[dev & 31][K];
+  if (__atomic_load_n(&li.ready, __ATOMIC_ACQUIRE)) {
+    out = li;
+    return cudaSuccess;
+  }
+  if (smem_max > 48 * 1024) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_max));
+    if (e != cudaSuccess) return e;
+  }
+  int sms = 0, occ = 0;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, smem)) !=
+      cudaSuccess)
+    return e;
+  li.sms = sms;
+  li.ctas_per_sm = occ > 0 ? occ : 1;
+  __atomic_store_n(&li.ready, 1, __ATOMIC_RELEASE);
+  out = li;
+  return cudaSuccess;
+}
+
+template <int D, bool BF16, bool KDA>
+cudaError_t decode_t(const KParams &p, cudaStream_t st) {
+  static LaunchInfo cache[32][kMaxComp + 1];
+  using L = SL<D, BF16, KDA>;
+  using TR = DecodeTraits<D, BF16, KDA>;
+  constexpr int NST = TR::kStages;
+  constexpr size_t scratch = sizeof(Scratch<D, !TR::kKtOverCodes>);
+  const size_t smem = NST * L(p.L.bytes).bytes + scratch;
+  const size_t smem_max = NST * L(record_layout(D, kMaxComp).bytes).bytes + scratch;
+  LaunchInfo li;
+  cudaError_t e = prepare(decode_kernel<D, BF16, KDA>, smem, smem_max, p.K, cache, li);
+  if (e != cudaSuccess) return e;
+  const int tiles = p.B * p.Hv;
+  int grid = li.sms * li.ctas_per_sm;
+  if (grid > tiles) grid = tiles;
+  const int need = (tiles + kMaxTilesPerCta - 1) / kMaxTilesPerCta;
+  if (grid < need) grid = need;
+  decode_kernel<D, BF16, KDA><<<grid, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D, bool BF16, bool KDA, int MODE>
+cudaError_t fold_t(const KParams &p, cudaStream_t st) {
+  static LaunchInfo cache[32][kMaxComp + 1];
+  using L = SL<D, BF16, KDA>;
+  const size_t smem = L(p.L.bytes).bytes + sizeof(Scratch<D, true>);
+  const size_t smem_max = L(record_layout(D, kMaxComp).bytes).bytes + sizeof(Scratch<D, true>);
+  LaunchInfo li;
+  cudaError_t e = prepare(fold_kernel<D, BF16, KDA, MODE>, smem, smem_max, p.K, cache, li);
+  if (e != cudaSuccess) return e;
+  fold_kernel<D, BF16, KDA, MODE><<<p.B * p.Hv, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t init_t(const KParams &p, cudaStream_t st) {
+  static LaunchInfo cache[32][kMaxComp + 1];
+  const size_t smem = D * D + sizeof(Scratch<D, false>);
+  LaunchInfo li;
+  cudaError_t e = prepare(init_kernel<D>, smem, smem, p.K, cache, li);
+  if (e != cudaSuccess) return e;
+  init_kernel<D><<<p.B * p.Hv, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <template <int, bool, bool> class F>
+cudaError_t dispatch3(const KParams &p, cudaStream_t s) {
+  const bool bf = p.in_bf16 != 0, kda = p.gate != 0;
+#define LQ_CASE(DD)                                     \
+  if (p.d == DD) {                                      \
+    if (bf && kda) return F<DD, true, true>::run(p, s); \
+    if (bf) return F<DD, true, false>::run(p, s);       \
+    if (kda) return F<DD, false, true>::run(p, s);      \
+    return F<DD, false, false>::run(p, s);              \
+  }
+  LQ_CASE(32)
+  LQ_CASE(64)
+  LQ_CASE(128)
+#undef LQ_CASE
+  return cudaErrorInvalidValue;
+}
+
+template <int D, bool BF, bool KDA>
+struct DecodeF {
+  static cudaError_t run(const KParams &p, cudaStream_t s) { return decode_t<D, BF, KDA>(p, s); }
+};
+template <int D, bool BF, bool KDA>
+struct FlushF {
+  static cudaError_t run(const KParams &p, cudaStream_t s) { return fold_t<D, BF, KDA, 0>(p, s); }
+};
+template <int D, bool BF, bool KDA>
+struct DequantF {
+  static cudaError_t run(const KParams &p, cudaStream_t s) { return fold_t<D, BF, KDA, 1>(p, s); }
+};
+
+}  // namespace
+
+cudaError_t launch_decode(const KParams &p, cudaStream_t s) { return dispatch3<DecodeF>(p, s); }
+cudaError_t launch_flush(const KParams &p, cudaStream_t s) { return dispatch3<FlushF>(p, s); }
+cudaError_t launch_dequantize(const KParams &p, cudaStream_t s) {
+  return dispatch3<DequantF>(p, s);
+}
+cudaError_t launch_init(const KParams &p, cudaStream_t s) {
+  if (p.d == 32) return init_t<32>(p, s);
+  if (p.d == 64) return init_t<64>(p, s);
+  if (p.d == 128) return init_t<128>(p, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lq

@@ -1,5 +1,6 @@
-// Internal interface between the C ABI (lq_capi.cu) and the kernels
-// (lq_kernels.cu).  Not installed; callers use include/leapquant.h.
+// Internal interface between the C ABI (lq_capi.cu, lq_noalloc.cu) and the
+// kernels (lq_decode.cu, lq_fp32.cu).  Not installed; callers use
+// include/leapquant.h.
 #pragma once
 
 #include <cstddef>
@@ -11,7 +12,9 @@ namespace lq {
 
 constexpr int kMaxWindow = 16;  // W limit: one buffer slot per token of a window
 constexpr int kMaxComp = 8;     // K limit
-constexpr int kErrBadPhase = 1;  // device error bit: buf_n outside [0, W)
+constexpr int kGdnGateStride = 16;  // GDN gate buffer: 16 floats per tile (one 64-byte copy)
+constexpr int kErrBadPhase = 1;     // device error bit: buf_n outside [0, W)
+constexpr int kErrTimeout = 2;      // device error bit: a bounded wait on a copy expired
 
 // Byte layout of one tile record (see include/leapquant.h).
 struct RecLayout {

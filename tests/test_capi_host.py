@@ -106,5 +106,5 @@ def test_empty_batch_is_a_no_op(B):
 
 
 def test_status_strings(B):
-    for s in range(7):
+    for s in range(8):
         assert B.lq_status_string(s).startswith("LQ_")
