@@ -193,14 +193,18 @@ def _oracle_inputs(w: wl.Workload, tiles_b: int, T: int, seed: int):
     return S0, ti
 
 
-def run_oracle_sample(w: wl.Workload, seqs: int, seed: int = 1234) -> tuple[float, int, int]:
-    """Time the oracle on `seqs` sequences x all heads for one window
-    (init + W tokens incl. the fold).  Returns (seconds, tile_steps, threads)."""
+def run_oracle_sample(w: wl.Workload, seqs: int, windows: int = 1,
+                      seed: int = 1234) -> tuple[float, int, int]:
+    """Time the oracle on `seqs` sequences x all heads for `windows` consecutive
+    W-token windows (each incl. its fold), the state carried from one window to
+    the next.  Only the oracle's decode calls are timed: the records are built
+    and each window's inputs drawn outside the timed region.  Returns
+    (seconds, tile_steps, threads)."""
     import oracle
 
     cfg = oracle.Cfg(w.d, w.d, W=w.window, K=w.n_comp, gate=w.gate, quant=1, smooth=w.smooth)
     T = w.window
-    S0, ti = _oracle_inputs(w, seqs, T, seed)
+    S0, _ = _oracle_inputs(w, seqs, 1, seed)
     tiles = seqs * w.num_v_heads
     recs = [oracle.quantize(cfg, S0[t].astype(np.float64)) for t in range(tiles)]
     rec = {"Q": np.stack([r.Q for r in recs]), "sig": np.stack([r.sig for r in recs]),
@@ -209,30 +213,39 @@ def run_oracle_sample(w: wl.Workload, seqs: int, seed: int = 1234) -> tuple[floa
     ga = w.d if w.gate == wl.GATE_DIAG else 1
     buf = {"n": np.zeros(tiles, np.int32), "bk": np.zeros((tiles, w.window, w.d)),
            "bd": np.zeros((tiles, w.window, w.d)), "ba": np.zeros((tiles, w.window, ga))}
-    inp = {n: np.ascontiguousarray(getattr(ti, n), dtype=np.float64)
-           for n in ("q", "k", "v", "alpha", "beta")}
-    inp["o"] = np.zeros((T, seqs, w.num_v_heads, w.d))
     threads = len(os.sched_getaffinity(0))
-    t0 = time.perf_counter()
-    used = oracle.batch_run(cfg, seqs, w.num_k_heads, w.num_v_heads, T, rec, buf, inp,
-                            nthreads=threads)
-    dt = time.perf_counter() - t0
-    return dt, tiles * T, used
+    dt, used = 0.0, threads
+    for win in range(windows):
+        ti = wl.token_inputs(np.random.default_rng(seed + 7919 * (win + 1)), w, T, batch=seqs)
+        inp = {n: np.ascontiguousarray(getattr(ti, n), dtype=np.float64)
+               for n in ("q", "k", "v", "alpha", "beta")}
+        inp["o"] = np.zeros((T, seqs, w.num_v_heads, w.d))
+        t0 = time.perf_counter()
+        used = oracle.batch_run(cfg, seqs, w.num_k_heads, w.num_v_heads, T, rec, buf, inp,
+                                nthreads=threads)
+        dt += time.perf_counter() - t0
+    return dt, tiles * T * windows, used
 
 
-def calibrate_oracle_seqs(w: wl.Workload, target_s: float) -> int:
-    dt, ts, _ = run_oracle_sample(w, 1)
-    per_seq = max(dt, 1e-4)
-    return int(max(1, min(w.batch, math.floor(target_s / per_seq))))
+def oracle_sample_size(w: wl.Workload, target_s: float) -> tuple[int, int]:
+    """(sequences, windows) for about `target_s` seconds of oracle work: first
+    more sequences (up to the batch), then more windows."""
+    dt1, _, _ = run_oracle_sample(w, 1)
+    per_seq = max(dt1, 1e-4)
+    seqs = int(max(1, min(w.batch, math.floor(target_s / per_seq))))
+    if seqs < w.batch:
+        return seqs, 1
+    dtb, _, _ = run_oracle_sample(w, seqs)
+    return seqs, int(max(1, math.floor(target_s / max(dtb, 1e-4))))
 
 
 def cpu_baseline(w: wl.Workload, target_s: float = 15.0) -> dict:
-    seqs = calibrate_oracle_seqs(w, target_s)
-    dt, ts, used = run_oracle_sample(w, seqs)
+    seqs, windows = oracle_sample_size(w, target_s)
+    dt, ts, used = run_oracle_sample(w, seqs, windows)
     return {"value": ts / dt, "unit": UNIT, "cores": used, "kind": "oracle",
-            "sample": (f"{seqs} of {w.batch} sequences x {w.num_v_heads} heads, one "
-                       f"{w.window}-token window incl. the fold, one layer; fp64 C oracle, "
-                       f"OpenMP over tiles; {dt:.1f} s")}
+            "sample": (f"{seqs} of {w.batch} sequences x {w.num_v_heads} heads, {windows} "
+                       f"consecutive {w.window}-token windows incl. their folds, one layer; "
+                       f"fp64 C oracle, OpenMP over tiles; {dt:.1f} s of oracle time")}
 
 
 def reference_arm(args, w: wl.Workload, rank: int, world: int) -> None:
@@ -240,13 +253,12 @@ def reference_arm(args, w: wl.Workload, rank: int, world: int) -> None:
         return
     steps, warm = args.steps, args.warmup
     budget = 150.0
-    dt1, ts1, _ = run_oracle_sample(w, 1)
-    seqs = int(max(1, min(w.batch, math.floor(budget / (steps + warm) / max(dt1, 1e-4)))))
+    seqs, windows = oracle_sample_size(w, budget / (steps + warm))
     for _ in range(warm):
-        run_oracle_sample(w, seqs)
+        run_oracle_sample(w, seqs, windows)
     tot_t, tot_ts, used = 0.0, 0, 1
     for s in range(steps):
-        dt, ts, used = run_oracle_sample(w, seqs, seed=1234 + s)
+        dt, ts, used = run_oracle_sample(w, seqs, windows, seed=1234 + s)
         tot_t += dt
         tot_ts += ts
     value = tot_ts / tot_t
@@ -256,8 +268,8 @@ def reference_arm(args, w: wl.Workload, rank: int, world: int) -> None:
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, args.layers),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
-                         "sample": (f"per step: {seqs} sequences x {w.num_v_heads} heads, one "
-                                    f"{w.window}-token window incl. the fold")},
+                         "sample": (f"per step: {seqs} sequences x {w.num_v_heads} heads, "
+                                    f"{windows} {w.window}-token window(s) incl. the fold")},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -311,6 +323,33 @@ class Layer:
                                    device=self.out.device)
 
 
+# ---------------------------------------------------------------------------
+# Ranks: one process per GPU, each on its own sequences (weak scaling)
+# ---------------------------------------------------------------------------
+
+def layer_seed(rank: int, layer: int) -> int:
+    """Seed of one rank's layer: every rank decodes its own sequences, so the
+    ranks share no data and the path needs no collective."""
+    return 1000 * rank + layer
+
+
+def max_over_ranks(x: float, world: int, device="cpu") -> float:
+    """Largest `x` over all ranks (the job takes as long as its slowest rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step: int, world: int, steps: int, ms_max: float) -> float:
+    """Units all ranks processed per second, over the slowest rank's time."""
+    return world * units_per_step * steps / (ms_max / 1e3)
+
+
 def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> None:
     import torch
     import torch.distributed as dist
@@ -320,7 +359,7 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     L = args.layers
-    layers = [Layer(B, w, seed=1000 * rank + l, device=device) for l in range(L)]
+    layers = [Layer(B, w, seed=layer_seed(rank, l), device=device) for l in range(L)]
     stream = torch.cuda.Stream(device=device)
     W = w.window
     launches_per_step = W * L
@@ -350,13 +389,6 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
     def barrier():
         if world > 1:
             dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     def timed(graph, steps, warmup, sample_clocks=False):
         with torch.cuda.stream(stream):
@@ -390,7 +422,7 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
             sampler.window(wall0, wall1)
         barrier()
         torch.cuda.synchronize()
-        ms = max_over_ranks(start.elapsed_time(end))
+        ms = max_over_ranks(start.elapsed_time(end), world, device)
         return ms, (sampler.summary() if sample_clocks else None)
 
     g8 = capture(step_int8)
@@ -405,8 +437,8 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
     del g32
 
     units_per_step = w.tiles * W * L               # per rank
-    value = world * units_per_step * args.steps / (ms8 / 1e3)
-    value32 = world * units_per_step * steps32 / (ms32 / 1e3)
+    value = whole_job_rate(units_per_step, world, args.steps, ms8)
+    value32 = whole_job_rate(units_per_step, world, steps32, ms32)
     ms_per_step = ms8 / args.steps
 
     # roofline of the decode kernel (algorithmic bytes / graph time per launch)
@@ -455,8 +487,8 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
         end.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms_e2e = max_over_ranks(start.elapsed_time(end))
-        e2e = {"value": world * units_per_step * e2e_steps / (ms_e2e / 1e3), "unit": UNIT,
+        ms_e2e = max_over_ranks(start.elapsed_time(end), world, device)
+        e2e = {"value": whole_job_rate(units_per_step, world, e2e_steps, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "path": "lq_decode_step_host (pinned host q,k,v,alpha,beta in; o out)"}
 

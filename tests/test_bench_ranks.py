@@ -1,0 +1,78 @@
+"""Multi-rank host logic of bench.py on CPU: two gloo ranks (one process per
+rank, as torchrun starts them) check the max-over-ranks timing, the whole-job
+rate, the per-rank seeds and that only rank 0 runs and prints the oracle arm.
+The decode path itself shards by sequence and has no collective."""
+import io
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, results):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    import datetime
+
+    import bench
+
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = [3.5, 7.25][rank]                       # per-rank device times
+        got = bench.max_over_ranks(ms, world, "cpu")
+        rate = bench.whole_job_rate(1000, world, 10, got)
+        seeds = [bench.layer_seed(rank, l) for l in range(8)]
+        gathered = [None] * world
+        dist.all_gather_object(gathered, seeds)
+        out = io.StringIO()
+        if rank != 0:
+            class Args:
+                steps, warmup, layers = 2, 3, 8
+            with redirect_stdout(out):
+                bench.reference_arm(Args, bench.WORKLOADS["qwen35_9b_gdn"], rank, world)
+        dist.barrier()
+        results[rank] = (got, rate, gathered, out.getvalue())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks():
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        mp.start_processes(_rank_main, args=(world, _free_port(), results), nprocs=world,
+                           join=True, start_method="spawn")
+        res = dict(results)
+    assert sorted(res) == [0, 1]
+    for rank in range(world):
+        got, rate, gathered, printed = res[rank]
+        assert got == 7.25                             # the slowest rank's time
+        assert rate == pytest.approx(2 * 1000 * 10 / 7.25e-3)
+        flat = [s for seeds in gathered for s in seeds]
+        assert len(set(flat)) == len(flat)             # no two ranks share a layer's data
+    assert res[1][3] == ""                             # rank 1 prints nothing
+
+
+def test_single_rank_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert not dist.is_initialized()
+    assert bench.max_over_ranks(4.0, 1) == 4.0
+    assert bench.whole_job_rate(5, 1, 2, 1000.0) == pytest.approx(10.0)
