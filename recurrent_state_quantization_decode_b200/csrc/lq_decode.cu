@@ -27,11 +27,15 @@
 //    product up to the digits' truncation (<= 7.5e-9 max|x| per element) and
 //    one rounding per combination step.  No code is ever converted to float on
 //    this path.
-//  * GDN with bf16 inputs takes a shorter per-token path: one warp does all
-//    per-channel work (gate product, x, digits, compensator dots) with no CTA
-//    barrier between the max and the digits, one warp gets the buffer
-//    coefficients c_s = rho_s k_s . k and a_s = rho_s k_s . q from a bf16
-//    m16n8k16 product, and the other row warps fetch their codes meanwhile.
+//  * GDN with bf16 inputs takes a shorter per-token path with one CTA barrier
+//    per tile.  Each int8 k-chunk (32 key channels) has its own digit scale,
+//    so one warp per chunk does that chunk's per-channel work (gate product, x,
+//    its max, digits, compensator dots) without a CTA-wide max; one warp gets
+//    the buffer coefficients c_s = rho_s k_s . k and a_s = rho_s k_s . q from a
+//    bf16 m16n8k16 product; the other row warps fetch their codes meanwhile.
+//    The per-token values are double-buffered, so a warp may start the next
+//    tile while others finish the current one, and every thread waits on the
+//    slot's mbarrier itself.
 //  * On the boundary token the fp32 state S = S0 diag(Gamma) + sum d_s kt_s^T
 //    is built in registers, in the same fragment layout as the codes, and the
 //    quantizer (compensator lines, smoothing, per-row int8) runs on it.
@@ -130,6 +134,7 @@ struct DecodeTraits {
   static constexpr bool kFast = BF16 && !KDA;
   static constexpr bool kKtOverCodes = kFast && kMaxWindow * FG<D>::PADW * 4 <= D * D;
   static constexpr int kStages = kFast ? 3 : 2;
+  static constexpr int kTok = kFast ? 2 : 1;  // per-token scratch buffers
 };
 
 // The scaled-key array lives in the scratch unless the decode kernel keeps it
@@ -141,27 +146,34 @@ struct KtArea {
 template <int D>
 struct KtArea<D, false> {};
 
-template <int D, bool KT>
-struct Scratch : KtArea<D, KT> {
+// Per-token values that the row phase reads: written before the tile's CTA
+// barrier, read after it.  The decode kernel for GDN with bf16 inputs keeps two
+// of these, so that one tile's per-channel work can overlap the previous
+// tile's row phase.
+template <int D>
+struct Tok {
   alignas(16) float qf[D];
   alignas(16) float kf[D];
   alignas(16) float vf[D];
   alignas(16) float G[D];                          // window gate Gamma per key channel
   alignas(16) float mG[FG<D>::PADW];               // m o Gamma
-  alignas(16) float invm[FG<D>::PADW];             // 1 / m (new smoothing factors)
   alignas(16) int8_t dig[8][FG<D>::DIGW];          // digits: rows 0-3 of x_q, 4-7 of x_k
-  alignas(16) float yq[D];
-  alignas(16) float yk[D];
-  alignas(16) float line[D];                       // the compensator line being extracted
-  alignas(16) double rowE[D];
   float cc[kMaxWindow + 1];
   float aa[kMaxWindow + 1];
   float cpart[kMaxComp][kWarps][2];  // per-warp partial row-compensator dots
   float rho[kMaxWindow + 1];         // scalar decay ratios (GDN)
+  float xmax[2][kWarps];
+  float xscale[2][4];  // digit scales of x_q, x_k (per int8 k-chunk on the GDN-bf16 path)
+};
+
+template <int D, bool KT, int NT = 1>
+struct Scratch : KtArea<D, KT> {
+  Tok<D> tok[NT];
+  alignas(16) float invm[FG<D>::PADW];             // 1 / m (new smoothing factors)
+  alignas(16) float line[D];                       // the compensator line being extracted
+  alignas(16) double rowE[D];
   double pbest[kWarps];              // per-warp partial argmax of the line energies
   int pid[kWarps];
-  float xmax[2][kWarps];
-  float xscale[2];
   int abort;
   int warp_cnt[kWarps];
   int tl_tile[kMaxTilesPerCta];
@@ -416,9 +428,9 @@ __device__ __forceinline__ void load_codes(const uint8_t *codes, uint4 (&A)[2][F
 //   S_ij = sigma_i code_ij (m_j Gamma_j) + sum_{s < nent} d_s[i] kt_s[j]
 //          + Gamma_j * (compensator lines),
 // with kt_s = k_s o (decay ratio to the last token) in kt (rows of PADW) and m o Gamma in
-// s.mG.  rsig, rcv, rcid point at the staged record; bd at the staged deltas.
+// x.mG.  rsig, rcv, rcid point at the staged record; bd at the staged deltas.
 template <int D, class SC>
-__device__ __forceinline__ void build_state(const SC &s, const float *kt,
+__device__ __forceinline__ void build_state(const SC &x, const float *kt,
                                             const uint4 (&A)[2][FG<D>::NSPAN],
                                             const float *rsig, const float *rcv, const int *rcid,
                                             const float *bd, int nent, int K,
@@ -431,7 +443,7 @@ __device__ __forceinline__ void build_state(const SC &s, const float *kt,
 #pragma unroll
   for (int h = 0; h < G::NSPAN; ++h) {
     if (chunk_valid<D>(t)) {
-      const float4 *mg4 = reinterpret_cast<const float4 *>(&s.mG[padc(frag_col(h, t, 0))]);
+      const float4 *mg4 = reinterpret_cast<const float4 *>(&x.mG[padc(frag_col(h, t, 0))]);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const float4 m = mg4[u];
@@ -482,14 +494,14 @@ __device__ __forceinline__ void build_state(const SC &s, const float *kt,
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int col = frag_col(h, t, e);
-            const float add = rcv[c * D + col] * s.G[col];
+            const float add = rcv[c * D + col] * x.G[col];
             if (second) SX(1, h, e) += add; else SX(0, h, e) += add;
           }
       }
     } else {
       const int jc = id - D;
       if (((jc & 63) >> 4) == t && chunk_valid<D>(t)) {
-        const float gj = s.G[jc];
+        const float gj = x.G[jc];
         const float a0 = rcv[c * D + r0] * gj, a1 = rcv[c * D + r1] * gj;
 #pragma unroll
         for (int h = 0; h < G::NSPAN; ++h)
@@ -808,11 +820,12 @@ __device__ __forceinline__ void issue_rest(const KParams &p, uint8_t *slot,
 // the lanes (lane s holds alpha_s).  Writes c_s = rho_s (k_s . k_t) and
 // a_s = rho_s (k_s . q_t) for s < n, a_n = k_t . q_t, and rho_s for s <= n.
 template <int D, class SC>
-__device__ __forceinline__ void coef_mma(SC &s, const __nv_bfloat16 *sbk,
+__device__ __forceinline__ void coef_mma(SC &x, const __nv_bfloat16 *sbk,
                                          const __nv_bfloat16 *sk, const __nv_bfloat16 *sq,
                                          const float *sbg, float alpha0, int n) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  // two independent accumulation chains (even / odd k16 steps), added at the end
+  float c[4] = {0.0f, 0.0f, 0.0f, 0.0f}, c2[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   const __nv_bfloat16 *row0 = (g < n) ? sbk + g * D : (g == n ? sk : nullptr);
   const __nv_bfloat16 *row1 = (g + 8 < n) ? sbk + (g + 8) * D : (g + 8 == n ? sk : nullptr);
   const __nv_bfloat16 *vec = (g == 0) ? sk : (g == 1 ? sq : nullptr);
@@ -824,8 +837,10 @@ __device__ __forceinline__ void coef_mma(SC &s, const __nv_bfloat16 *sbk,
     const uint4 a1 = row1 ? *reinterpret_cast<const uint4 *>(row1 + off) : zero;
     const uint4 bb = vec ? *reinterpret_cast<const uint4 *>(vec + off) : zero;
     mma_bf16(c, a0.x, a1.x, a0.y, a1.y, bb.x, bb.y);
-    mma_bf16(c, a0.z, a1.z, a0.w, a1.w, bb.z, bb.w);
+    mma_bf16(c2, a0.z, a1.z, a0.w, a1.w, bb.z, bb.w);
   }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) c[e] += c2[e];
   float P = (lane < n) ? sbg[lane] : (lane == n ? alpha0 : 1.0f);
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -837,14 +852,14 @@ __device__ __forceinline__ void coef_mma(SC &s, const __nv_bfloat16 *sbk,
   const float rho1 = __shfl_sync(kFull, P, (g + 9) & 31);
   if (t == 0) {
     if (g <= n) {
-      s.cc[g] = rho0 * c[0];
-      s.aa[g] = rho0 * c[1];
-      s.rho[g] = rho0;
+      x.cc[g] = rho0 * c[0];
+      x.aa[g] = rho0 * c[1];
+      x.rho[g] = rho0;
     }
     if (g + 8 <= n) {
-      s.cc[g + 8] = rho1 * c[2];
-      s.aa[g + 8] = rho1 * c[3];
-      s.rho[g + 8] = rho1;
+      x.cc[g + 8] = rho1 * c[2];
+      x.aa[g + 8] = rho1 * c[3];
+      x.rho[g + 8] = rho1;
     }
   }
 }
@@ -874,98 +889,76 @@ __device__ __forceinline__ void digit_scales(float M, float &up, float &down) {
   }
 }
 
-// GDN with bf16 inputs: all per-channel work of a tile in one warp; lane l
-// takes the CPL = D/32 consecutive channels CPL*l ... CPL*l + CPL-1.  Writes
-// q, k, v (fp32), Gamma, m o Gamma, the digits of x_q and x_k with their
-// scales, the row-compensator partial dots (cpart[c][0]), and appends k_t.
-template <int D, class SC>
-__device__ __forceinline__ void channel_warp_fast(const KParams &p, SC &s,
-                                                  const __nv_bfloat16 *sq,
-                                                  const __nv_bfloat16 *sk,
-                                                  const __nv_bfloat16 *sv, const float *sbg,
-                                                  const float *rm, const float *rcv,
-                                                  const int *rcid, float alpha0, int n,
-                                                  size_t key_slot, bool writes_key) {
-  constexpr int CPL = D / 32;
+// GDN with bf16 inputs: warp c < 2 * NSPAN does the per-channel work of int8
+// MMA k-chunk c, the 32 columns 64h + 16t + 8u + e (h = c / 2, u = c % 2,
+// t < 4, e < 8) that the chunk's codes cover; lane l takes t = l / 8, e = l % 8.
+// Each chunk's digits get their own power-of-two scale, so the max is a warp
+// reduction.  Writes q, k, v (fp32), Gamma, m o Gamma, the chunk's digits and
+// scales and its partial row-compensator dots (cpart[line][c]); warp 0 also
+// appends k_t.
+template <int D, class TK>
+__device__ __forceinline__ void channel_chunk_fast(const KParams &p, TK &x,
+                                                   const __nv_bfloat16 *sq,
+                                                   const __nv_bfloat16 *sk,
+                                                   const __nv_bfloat16 *sv, const float *sbg,
+                                                   const float *rm, const float *rcv,
+                                                   const int *rcid, float alpha0, int n,
+                                                   size_t key_slot, bool writes_key, int c) {
   const int lane = threadIdx.x & 31;
-  const int j0 = CPL * lane;
+  const int tq = lane >> 3;
+  const int j = 64 * (c >> 1) + 16 * tq + 8 * (c & 1) + (lane & 7);
+  const bool valid = D >= 64 || tq < 2;
   // window gate Gamma_t = prod of the n buffered gates and the current one
   float P = (lane < n) ? sbg[lane] : (lane == n ? alpha0 : 1.0f);
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) P *= __shfl_xor_sync(kFull, P, o);
   const float Gm = P;
-  float q[CPL], k[CPL], xq[CPL], xk[CPL];
-  float mq = 0.0f, mk = 0.0f;
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) {
-    const int j = j0 + c;
-    q[c] = __bfloat162float(sq[j]);
-    k[c] = __bfloat162float(sk[j]);
+  float q = 0.0f, k = 0.0f, xq = 0.0f, xk = 0.0f;
+  if (valid) {
+    q = __bfloat162float(sq[j]);
+    k = __bfloat162float(sk[j]);
     const float mj = rm[j];
-    s.qf[j] = q[c];
-    s.kf[j] = k[c];
-    s.vf[j] = __bfloat162float(sv[j]);
-    s.G[j] = Gm;
-    s.mG[padc(j)] = mj * Gm;
-    xq[c] = mj * (Gm * q[c]);
-    xk[c] = mj * (Gm * k[c]);
-    mq = fmaxf(mq, fabsf(xq[c]));
-    mk = fmaxf(mk, fabsf(xk[c]));
+    x.qf[j] = q;
+    x.kf[j] = k;
+    x.vf[j] = __bfloat162float(sv[j]);
+    x.G[j] = Gm;
+    x.mG[padc(j)] = mj * Gm;
+    xq = mj * (Gm * q);
+    xk = mj * (Gm * k);
+    if (writes_key) reinterpret_cast<__nv_bfloat16 *>(p.buf_k)[key_slot + j] = sk[j];
   }
-  if (writes_key) {
-    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.buf_k) + key_slot;
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) dst[j0 + c] = sk[j0 + c];
-  }
-  mq = warp_max_abs(mq);
-  mk = warp_max_abs(mk);
+  const float mq = warp_max_abs(xq), mk = warp_max_abs(xk);
   float upq = 0.0f, dnq = 0.0f, upk = 0.0f, dnk = 0.0f;
   if (mq > 0.0f) digit_scales(mq, upq, dnq);
   if (mk > 0.0f) digit_scales(mk, upk, dnk);
   uint32_t dq[4] = {0u, 0u, 0u, 0u}, dk[4] = {0u, 0u, 0u, 0u};
+  digits4(xq * upq, dq, 0);
+  digits4(xk * upk, dk, 0);
+  if (valid) {
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) {
-    digits4(xq[c] * upq, dq, 8 * c);
-    digits4(xk[c] * upk, dk, 8 * c);
-  }
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    if constexpr (CPL == 4) {
-      *reinterpret_cast<uint32_t *>(&s.dig[r][j0]) = dq[r];
-      *reinterpret_cast<uint32_t *>(&s.dig[4 + r][j0]) = dk[r];
-    } else {
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        s.dig[r][j0 + c] = static_cast<int8_t>((dq[r] >> (8 * c)) & 0xffu);
-        s.dig[4 + r][j0 + c] = static_cast<int8_t>((dk[r] >> (8 * c)) & 0xffu);
-      }
+    for (int r = 0; r < 4; ++r) {
+      x.dig[r][j] = static_cast<int8_t>(dq[r]);
+      x.dig[4 + r][j] = static_cast<int8_t>(dk[r]);
     }
   }
   if (lane == 0) {
-    s.xscale[0] = dnq;
-    s.xscale[1] = dnk;
+    x.xscale[0][c] = dnq;
+    x.xscale[1][c] = dnk;
   }
-  // row-compensator lines dotted with Gamma o q and Gamma o k
+  // row-compensator lines dotted with Gamma o q and Gamma o k over this chunk
+  const float gq = Gm * q, gk = Gm * k;
   for (int c0 = 0; c0 < p.K; c0 += 4) {
     float v[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int c = c0 + i;
-      float aq = 0.0f, ak = 0.0f;
-      if (c < p.K && rcid[c] < D) {
-#pragma unroll
-        for (int u = 0; u < CPL; ++u) {
-          const float cvj = rcv[c * D + j0 + u];
-          aq = fmaf(cvj, q[u], aq);
-          ak = fmaf(cvj, k[u], ak);
-        }
-      }
-      v[2 * i] = Gm * aq;
-      v[2 * i + 1] = Gm * ak;
+      const int line = c0 + i;
+      const float cvj = (valid && line < p.K && rcid[line] < D) ? rcv[line * D + j] : 0.0f;
+      v[2 * i] = cvj * gq;
+      v[2 * i + 1] = cvj * gk;
     }
     const float tot = warp_sum8(v, lane);
-    const int vi = (lane >> 2) & 7, c = c0 + (vi >> 1);
-    if ((lane & 3) == 0 && c < p.K) s.cpart[c][0][vi & 1] = tot;
+    const int vi = (lane >> 2) & 7, line = c0 + (vi >> 1);
+    if ((lane & 3) == 0 && line < p.K) x.cpart[line][c][vi & 1] = tot;
   }
 }
 
@@ -980,10 +973,10 @@ __device__ __forceinline__ void channel_warp_fast(const KParams &p, SC &s,
 //  C  every row warp: y_q, y_k for its 16 rows on the int8 tensor path, then
 //     finishes its rows (buffer sums split over the 4 lanes of a row):
 //     d_t = beta (v - y_k - sum c_s d_s), o_t = y_q + sum a_s d_s + a_t d_t.
-template <int D, bool BF16, bool KDA, class SC>
-__device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *slot,
+template <int D, bool BF16, bool KDA, class SC, class Refill>
+__device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x, uint8_t *slot,
                                              int tile, int n, int coord, float alpha0,
-                                             float beta) {
+                                             float beta, Refill &&refill) {
   using G = FG<D>;
   using L = SL<D, BF16, KDA>;
   using IT = in_t<BF16>;
@@ -1008,35 +1001,42 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
 
   // ---- Phases A and B ----
   constexpr bool kFast = DecodeTraits<D, BF16, KDA>::kFast;
-  constexpr int CWP = kFast ? 1 : CW;  // warps holding compensator partial dots
+  constexpr int NCH = 2 * G::NSPAN;    // int8 MMA k-chunks (GDN-bf16: one channel warp each)
+  constexpr int CWP = kFast ? NCH : CW;  // warps holding compensator partial dots
   uint4 A[2][G::NSPAN];
   if constexpr (kFast) {
-    // one warp for the channels, one for the buffer coefficients; the other
-    // row warps fetch their code fragments
-    if (warp == 0) {
-      channel_warp_fast<D>(p, s, reinterpret_cast<const __nv_bfloat16 *>(sq),
-                           reinterpret_cast<const __nv_bfloat16 *>(sk),
-                           reinterpret_cast<const __nv_bfloat16 *>(sv), sbg, rm, rcv, rcid,
-                           alpha0, n,
-                           ((static_cast<size_t>(b) * p.Hk + hk) * p.W + n) * D, writes_key);
-      if (lane == 0) p.buf_g[static_cast<size_t>(tile) * kGdnGateStride + n] = alpha0;
-    } else if (warp == 1) {
-      coef_mma<D>(s, reinterpret_cast<const __nv_bfloat16 *>(sbk),
+    // one warp per k-chunk for the channels, one for the buffer coefficients;
+    // the other row warps fetch their code fragments
+    if (warp < NCH) {
+      if (warp < G::NRB) load_codes<D>(codes, A);
+      channel_chunk_fast<D>(p, x, reinterpret_cast<const __nv_bfloat16 *>(sq),
+                            reinterpret_cast<const __nv_bfloat16 *>(sk),
+                            reinterpret_cast<const __nv_bfloat16 *>(sv), sbg, rm, rcv, rcid,
+                            alpha0, n,
+                            ((static_cast<size_t>(b) * p.Hk + hk) * p.W + n) * D, writes_key,
+                            warp);
+      if (tid == 0) p.buf_g[static_cast<size_t>(tile) * kGdnGateStride + n] = alpha0;
+    } else if (warp == NCH) {
+      coef_mma<D>(x, reinterpret_cast<const __nv_bfloat16 *>(sbk),
                   reinterpret_cast<const __nv_bfloat16 *>(sk),
                   reinterpret_cast<const __nv_bfloat16 *>(sq), sbg, alpha0, n);
     } else if (warp < G::NRB) {
       load_codes<D>(codes, A);
     }
+    // the one CTA barrier of a plain token: the copies of this tile have
+    // landed for every thread, and the previous tile's slot is free
     __syncthreads();
+    if (s.abort) return false;
+    refill();
   } else {
     // ---- Phase A ----
   float xq = 0.0f, xk = 0.0f;
   if (tid < D) {
     const int j = tid;
     const float qj = to_f(sq[j]), kj = to_f(sk[j]);
-    s.qf[j] = qj;
-    s.kf[j] = kj;
-    s.vf[j] = to_f(sv[j]);
+    x.qf[j] = qj;
+    x.kf[j] = kj;
+    x.vf[j] = to_f(sv[j]);
     float acc;
     if constexpr (kFast) {
       // window gate Gamma_t = prod of the n buffered gates and the current one
@@ -1054,19 +1054,19 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
       }
       s.kt[n][padc(j)] = kj;
     }
-    s.G[j] = acc;
+    x.G[j] = acc;
     const float mj = rm[j];
     xq = mj * (acc * qj);
     xk = mj * (acc * kj);
-    s.mG[padc(j)] = mj * acc;
+    x.mG[padc(j)] = mj * acc;
     if (writes_key)
       reinterpret_cast<IT *>(p.buf_k)[((static_cast<size_t>(b) * p.Hk + hk) * p.W + n) * D + j] =
           sk[j];
     if constexpr (KDA) p.buf_g[(static_cast<size_t>(tile) * p.W + n) * D + j] = sa[j];
     const float mq = warp_max_abs(xq), mk = warp_max_abs(xk);
     if (lane == 0) {
-      s.xmax[0][warp] = mq;
-      s.xmax[1][warp] = mk;
+      x.xmax[0][warp] = mq;
+      x.xmax[1][warp] = mk;
     }
     // row-compensator lines dotted with Gamma o q and Gamma o k: per-warp
     // partials, four lines per transposed reduction
@@ -1082,13 +1082,13 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
       }
       const float tot = warp_sum8(v, lane);
       const int vi = (lane >> 2) & 7, c = c0 + (vi >> 1);
-      if ((lane & 3) == 0 && c < p.K) s.cpart[c][warp][vi & 1] = tot;
+      if ((lane & 3) == 0 && c < p.K) x.cpart[c][warp][vi & 1] = tot;
     }
   } else if (warp < G::NRB) {
     load_codes<D>(codes, A);
   }
   if constexpr (kFast) {
-    if (warp == CW) coef_mma<D>(s, reinterpret_cast<const __nv_bfloat16 *>(sbk),
+    if (warp == CW) coef_mma<D>(x, reinterpret_cast<const __nv_bfloat16 *>(sbk),
                                 reinterpret_cast<const __nv_bfloat16 *>(sk),
                                 reinterpret_cast<const __nv_bfloat16 *>(sq), sbg, alpha0, n);
   }
@@ -1102,14 +1102,14 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
     float Mq = 0.0f, Mk = 0.0f;
 #pragma unroll
     for (int w = 0; w < CW; ++w) {
-      Mq = fmaxf(Mq, s.xmax[0][w]);
-      Mk = fmaxf(Mk, s.xmax[1][w]);
+      Mq = fmaxf(Mq, x.xmax[0][w]);
+      Mk = fmaxf(Mk, x.xmax[1][w]);
     }
-    split_digits(xq, Mq, &s.dig[0][tid], G::DIGW);
-    split_digits(xk, Mk, &s.dig[4][tid], G::DIGW);
+    split_digits(xq, Mq, &x.dig[0][tid], G::DIGW);
+    split_digits(xk, Mk, &x.dig[4][tid], G::DIGW);
     if (tid == 0) {
-      s.xscale[0] = digit_scale(Mq);
-      s.xscale[1] = digit_scale(Mk);
+      x.xscale[0][0] = digit_scale(Mq);
+      x.xscale[1][0] = digit_scale(Mk);
     }
   } else if constexpr (!kFast) {
     // c_s = kt_s . k and a_s = kt_s . q for the buffered tokens; a_t = k . q
@@ -1117,8 +1117,8 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
       float c = 0.0f, a = 0.0f;
       for (int j = lane; j < D; j += 32) {
         const float kv = s.kt[sl][padc(j)];
-        c = fmaf(kv, s.kf[j], c);
-        a = fmaf(kv, s.qf[j], a);
+        c = fmaf(kv, x.kf[j], c);
+        a = fmaf(kv, x.qf[j], a);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
@@ -1126,8 +1126,8 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
         a += __shfl_xor_sync(kFull, a, o);
       }
       if (lane == 0) {
-        s.cc[sl] = c;
-        s.aa[sl] = a;
+        x.cc[sl] = c;
+        x.aa[sl] = a;
       }
     }
   }
@@ -1137,29 +1137,59 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
 
   // ---- Phase C ----
   if (warp < G::NRB) {
-    if (kFast ? warp < 2 : tid < D) load_codes<D>(codes, A);
-    int acc[4] = {0, 0, 0, 0};
-#pragma unroll
-    for (int hh = 0; hh < G::NSPAN; ++hh) {
-      uint4 Bw = make_uint4(0, 0, 0, 0);
-      if (chunk_valid<D>(t))
-        Bw = *reinterpret_cast<const uint4 *>(&s.dig[g][frag_col(hh, t, 0)]);
-      mma_s8(acc, A[0][hh].x, A[1][hh].x, A[0][hh].y, A[1][hh].y, Bw.x, Bw.y);
-      mma_s8(acc, A[0][hh].z, A[1][hh].z, A[0][hh].w, A[1][hh].w, Bw.z, Bw.w);
-    }
+    if (kFast ? warp == NCH : tid < D) load_codes<D>(codes, A);
     // lane (g, t) holds digits 2t, 2t+1 of rows r0 (acc 0,1) and r0+8 (acc 2,3);
     // t = 0,1: x_q digits 0-1, 2-3; t = 2,3: x_k digits 0-1, 2-3.
-    float p0 = static_cast<float>(acc[0]) + static_cast<float>(acc[1]) * (1.0f / 128.0f);
-    float p1 = static_cast<float>(acc[2]) + static_cast<float>(acc[3]) * (1.0f / 128.0f);
-    if (t & 1) {
-      p0 *= 1.0f / 16384.0f;
-      p1 *= 1.0f / 16384.0f;
+    float p0, p1, sq0, sk0;
+    if constexpr (kFast) {
+      // one accumulator per k-chunk, each with its own digit scale
+      int acc[NCH][4];
+#pragma unroll
+      for (int hh = 0; hh < G::NSPAN; ++hh) {
+        uint4 Bw = make_uint4(0, 0, 0, 0);
+        if (chunk_valid<D>(t))
+          Bw = *reinterpret_cast<const uint4 *>(&x.dig[g][frag_col(hh, t, 0)]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[2 * hh][e] = acc[2 * hh + 1][e] = 0;
+        mma_s8(acc[2 * hh], A[0][hh].x, A[1][hh].x, A[0][hh].y, A[1][hh].y, Bw.x, Bw.y);
+        mma_s8(acc[2 * hh + 1], A[0][hh].z, A[1][hh].z, A[0][hh].w, A[1][hh].w, Bw.z, Bw.w);
+      }
+      const float pair = (t & 1) ? 1.0f / 16384.0f : 1.0f;
+      p0 = 0.0f;
+      p1 = 0.0f;
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        const float sc = x.xscale[t >> 1][c] * pair;
+        p0 = fmaf(sc, static_cast<float>(acc[c][0]) +
+                          static_cast<float>(acc[c][1]) * (1.0f / 128.0f), p0);
+        p1 = fmaf(sc, static_cast<float>(acc[c][2]) +
+                          static_cast<float>(acc[c][3]) * (1.0f / 128.0f), p1);
+      }
+      sq0 = 1.0f;
+      sk0 = 1.0f;
+    } else {
+      int acc[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int hh = 0; hh < G::NSPAN; ++hh) {
+        uint4 Bw = make_uint4(0, 0, 0, 0);
+        if (chunk_valid<D>(t))
+          Bw = *reinterpret_cast<const uint4 *>(&x.dig[g][frag_col(hh, t, 0)]);
+        mma_s8(acc, A[0][hh].x, A[1][hh].x, A[0][hh].y, A[1][hh].y, Bw.x, Bw.y);
+        mma_s8(acc, A[0][hh].z, A[1][hh].z, A[0][hh].w, A[1][hh].w, Bw.z, Bw.w);
+      }
+      p0 = static_cast<float>(acc[0]) + static_cast<float>(acc[1]) * (1.0f / 128.0f);
+      p1 = static_cast<float>(acc[2]) + static_cast<float>(acc[3]) * (1.0f / 128.0f);
+      if (t & 1) {
+        p0 *= 1.0f / 16384.0f;
+        p1 *= 1.0f / 16384.0f;
+      }
+      sq0 = x.xscale[0][0];
+      sk0 = x.xscale[1][0];
     }
     p0 += __shfl_xor_sync(kFull, p0, 1);
     p1 += __shfl_xor_sync(kFull, p1, 1);
     const int r0 = 16 * warp + g, r1 = r0 + 8;
     const int base_lane = lane & ~3;
-    const float sq0 = s.xscale[0], sk0 = s.xscale[1];
     float yq0 = __shfl_sync(kFull, p0, base_lane) * sq0 * rsig[r0];
     float yq1 = __shfl_sync(kFull, p1, base_lane) * sq0 * rsig[r1];
     float yk0 = __shfl_sync(kFull, p0, base_lane | 2) * sk0 * rsig[r0];
@@ -1168,7 +1198,7 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
     // xa collects what adds to o, xc what is subtracted from v
     float xc0 = 0.0f, xa0 = 0.0f, xc1 = 0.0f, xa1 = 0.0f;
     for (int sl = t; sl < n; sl += 4) {
-      const float c = s.cc[sl], a = s.aa[sl];
+      const float c = x.cc[sl], a = x.aa[sl];
       const float d0 = sbd[sl * D + r0], d1 = sbd[sl * D + r1];
       xc0 = fmaf(c, d0, xc0);
       xa0 = fmaf(a, d0, xa0);
@@ -1182,8 +1212,8 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
           float dq = 0.0f, dk = 0.0f;
 #pragma unroll
           for (int w = 0; w < CWP; ++w) {
-            dq += s.cpart[c][w][0];
-            dk += s.cpart[c][w][1];
+            dq += x.cpart[c][w][0];
+            dk += x.cpart[c][w][1];
           }
           if (id == r0) {
             xa0 += dq;
@@ -1195,8 +1225,8 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
         }
       } else {
         const int jc = id - D;
-        const float gj = s.G[jc];
-        const float gq = gj * s.qf[jc], gk = gj * s.kf[jc];
+        const float gj = x.G[jc];
+        const float gq = gj * x.qf[jc], gk = gj * x.kf[jc];
         const float c0 = rcv[c * D + r0], c1 = rcv[c * D + r1];
         xa0 = fmaf(c0, gq, xa0);
         xc0 = fmaf(c0, gk, xc0);
@@ -1215,8 +1245,8 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
       const int row = t ? r1 : r0;
       const float yq = t ? yq1 : yq0, yk = t ? yk1 : yk0;
       const float xc = t ? xc1 : xc0, xa = t ? xa1 : xa0;
-      const float dt = beta * (s.vf[row] - yk - xc);
-      const float o = fmaf(s.aa[n], dt, yq + xa);
+      const float dt = beta * (x.vf[row] - yk - xc);
+      const float o = fmaf(x.aa[n], dt, yq + xa);
       st_out(p.out, static_cast<size_t>(tile) * D + row, o, p.out_bf16);
       p.buf_d[(static_cast<size_t>(tile) * p.W + n) * D + row] = dt;
       sbd[n * D + row] = dt;
@@ -1224,7 +1254,7 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
   }
   if (n + 1 < p.W) {
     if (tid == 0) p.buf_n[tile] = n + 1;
-    return;
+    return true;
   }
 
   // Window boundary: fold the W buffered tokens and requantize.
@@ -1245,20 +1275,21 @@ __device__ __forceinline__ void process_tile(const KParams &p, SC &s, uint8_t *s
     }
     if (tid < D) {
       for (int sl = 0; sl < n; ++sl)
-        ktw[sl * G::PADW + padc(tid)] = to_f(sbk[sl * D + tid]) * s.rho[sl];
-      ktw[n * G::PADW + padc(tid)] = s.kf[tid];
+        ktw[sl * G::PADW + padc(tid)] = to_f(sbk[sl * D + tid]) * x.rho[sl];
+      ktw[n * G::PADW + padc(tid)] = x.kf[tid];
     }
     __syncthreads();
     kt = ktw;
   } else {
     kt = &s.kt[0][0];
   }
-  if (warp < G::NRB) build_state<D>(s, kt, Af, rsig, rcv, rcid, sbd, n + 1, p.K, S);
+  if (warp < G::NRB) build_state<D>(x, kt, Af, rsig, rcv, rcid, sbd, n + 1, p.K, S);
   __syncthreads();  // the staged codes and keys are now free for the quantizer's scratch
   quantize_tile<D>(s, reinterpret_cast<double *>(slot + L::QS_COLPART),
                    reinterpret_cast<float *>(slot + L::QS_COLMAX), S,
                    p.records + static_cast<size_t>(tile) * p.L.bytes, p.L, p.K, p.smooth);
   if (tid == 0) p.buf_n[tile] = 0;
+  return true;
 }
 
 template <int D, bool BF16, bool KDA>
@@ -1266,7 +1297,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
   using L = SL<D, BF16, KDA>;
   using TR = DecodeTraits<D, BF16, KDA>;
   constexpr int kStages = TR::kStages;
-  using SC = Scratch<D, !TR::kKtOverCodes>;
+  using SC = Scratch<D, !TR::kKtOverCodes, TR::kTok>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int slot_bytes = L(p.L.bytes).bytes;
   SC &s = *reinterpret_cast<SC *>(smem + kStages * slot_bytes);
@@ -1332,26 +1363,55 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
       if (!speculate) issue_record<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[st]);
       issue_rest<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[st], s.tl_n[st], s.tl_coord[st]);
     }
+  // tiles whose copies have been issued (the same value in every thread)
+  int issued = count < kStages ? count : kStages;
+  auto refill = [&](int freed) {
+    // slot freed % kStages takes the next tile in line
+    if (freed >= 0 && issued < count) {
+      if (tid == 0) {
+        uint8_t *slot = smem + (freed % kStages) * slot_bytes;
+        const int nx = issued;
+        issue_record<D, BF16, KDA>(p, slot, &s.bar[freed % kStages], s.tl_tile[nx]);
+        issue_rest<D, BF16, KDA>(p, slot, &s.bar[freed % kStages], s.tl_tile[nx], s.tl_n[nx],
+                                 s.tl_coord[nx]);
+      }
+      ++issued;
+    }
+  };
 
   int i = 0;
   for (; i < count; ++i) {
     const int st = i % kStages;
     const uint32_t parity = static_cast<uint32_t>(i / kStages) & 1u;
-    if (!mbar_wait_bounded(&s.bar[st], parity)) s.abort = 1;
-    __syncthreads();
-    if (s.abort) break;
-    if (s.tl_n[i] >= 0)
-      process_tile<D, BF16, KDA>(p, s, smem + st * slot_bytes, s.tl_tile[i], s.tl_n[i],
-                                 s.tl_coord[i], s.tl_a[i], s.tl_b[i]);
-    // The slot was read and written through the generic proxy; order that
-    // before the bulk copy that refills it.
-    fence_proxy_async();
-    __syncthreads();
-    if (tid == 0 && i + kStages < count) {
-      const int nx = i + kStages;
-      uint8_t *slot = smem + st * slot_bytes;
-      issue_record<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[nx]);
-      issue_rest<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[nx], s.tl_n[nx], s.tl_coord[nx]);
+    if constexpr (TR::kTok == 2) {
+      // Every thread waits for the copies itself; the tile's one CTA barrier
+      // (inside process_tile) then makes the abort decision uniform and frees
+      // the previous tile's slot, which is refilled right after it.
+      if (!mbar_wait_bounded(&s.bar[st], parity)) s.abort = 1;
+      bool ok;
+      if (s.tl_n[i] >= 0) {
+        ok = process_tile<D, BF16, KDA>(p, s, s.tok[i & 1], smem + st * slot_bytes,
+                                        s.tl_tile[i], s.tl_n[i], s.tl_coord[i], s.tl_a[i],
+                                        s.tl_b[i], [&] { refill(i - 1); });
+      } else {
+        __syncthreads();
+        ok = !s.abort;
+        if (ok) refill(i - 1);
+      }
+      if (!ok) break;
+      // The slot was read and written through the generic proxy; order that
+      // before the bulk copy that will refill it.
+      fence_proxy_async();
+    } else {
+      if (!mbar_wait_bounded(&s.bar[st], parity)) s.abort = 1;
+      __syncthreads();
+      if (s.abort) break;
+      if (s.tl_n[i] >= 0)
+        process_tile<D, BF16, KDA>(p, s, s.tok[0], smem + st * slot_bytes, s.tl_tile[i],
+                                   s.tl_n[i], s.tl_coord[i], s.tl_a[i], s.tl_b[i], [] {});
+      fence_proxy_async();
+      __syncthreads();
+      refill(i);
     }
   }
   if (i < count) {
@@ -1359,8 +1419,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
     // flight into this CTA's shared memory a bounded chance to land.
     if (tid == 0) {
       atomicOr(p.err, kErrTimeout);
-      const int last = (i + kStages < count) ? i + kStages : count;
-      for (int k = i; k < last; ++k)
+      for (int k = i; k < issued; ++k)
         mbar_wait_bounded(&s.bar[k % kStages], static_cast<uint32_t>(k / kStages) & 1u);
     }
     __syncthreads();
@@ -1406,6 +1465,7 @@ __global__ void __launch_bounds__(kThreads) fold_kernel(const KParams p) {
   uint8_t *slot = smem;
   const L lay(p.L.bytes);
   Scratch<D, true> &s = *reinterpret_cast<Scratch<D, true> *>(smem + lay.bytes);
+  Tok<D> &x = s.tok[0];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int tile = blockIdx.x;
@@ -1434,15 +1494,15 @@ __global__ void __launch_bounds__(kThreads) fold_kernel(const KParams p) {
       s.kt[sl][padc(j)] = to_f(sbk[sl * D + j]) * acc;
       acc *= KDA ? sbg[sl * D + j] : sbg[sl];
     }
-    s.G[j] = acc;
-    s.mG[padc(j)] = rm[j] * acc;
+    x.G[j] = acc;
+    x.mG[padc(j)] = rm[j] * acc;
   }
   __syncthreads();
   float2 S[2][G::NSPAN][8];
   if (warp < G::NRB) {
     uint4 A[2][G::NSPAN];
     load_codes<D>(slot, A);
-    build_state<D>(s, &s.kt[0][0], A, rsig, rcv, rcid, sbd, n, p.K, S);
+    build_state<D>(x, &s.kt[0][0], A, rsig, rcv, rcid, sbd, n, p.K, S);
   }
   if constexpr (MODE == 0) {
     __syncthreads();
@@ -1554,7 +1614,7 @@ cudaError_t decode_t(const KParams &p, cudaStream_t st) {
   using L = SL<D, BF16, KDA>;
   using TR = DecodeTraits<D, BF16, KDA>;
   constexpr int NST = TR::kStages;
-  constexpr size_t scratch = sizeof(Scratch<D, !TR::kKtOverCodes>);
+  constexpr size_t scratch = sizeof(Scratch<D, !TR::kKtOverCodes, TR::kTok>);
   const size_t smem = NST * L(p.L.bytes).bytes + scratch;
   const size_t smem_max = NST * L(record_layout(D, kMaxComp).bytes).bytes + scratch;
   LaunchInfo li;
