@@ -175,6 +175,7 @@ struct Scratch : KtArea<D, KT> {
   double pbest[kWarps];              // per-warp partial argmax of the line energies
   int pid[kWarps];
   int abort;
+  int done[3];  // warps finished with each ring slot (GDN-bf16 path)
   int warp_cnt[kWarps];
   int tl_tile[kMaxTilesPerCta];
   int tl_n[kMaxTilesPerCta];      // window phase; -1: skip (corrupt phase)
@@ -1313,8 +1314,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
   const bool speculate = p.mask == nullptr;
   if (tid == 0) {
     s.abort = 0;
-    for (int st = 0; st < kStages; ++st) mbar_init(&s.bar[st], 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&s.bar[st], 1);
+      s.done[st] = 0;
+    }
     fence_mbar_init();
+  }
+  // Launched as a programmatic dependent: everything above touched only this
+  // CTA's shared memory.  Wait here until the previous kernel in the stream
+  // has completed and its writes are visible, and let the next one start
+  // its own setup as this grid's CTAs retire.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (tid == 0) {
     if (speculate)
       for (int st = 0; st < kStages && st < mine; ++st)
         issue_record<D, BF16, KDA>(p, smem + st * slot_bytes, &s.bar[st],
@@ -1392,16 +1404,32 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
       if (s.tl_n[i] >= 0) {
         ok = process_tile<D, BF16, KDA>(p, s, s.tok[i & 1], smem + st * slot_bytes,
                                         s.tl_tile[i], s.tl_n[i], s.tl_coord[i], s.tl_a[i],
-                                        s.tl_b[i], [&] { refill(i - 1); });
+                                        s.tl_b[i], [] {});
       } else {
         __syncthreads();
         ok = !s.abort;
-        if (ok) refill(i - 1);
       }
       if (!ok) break;
-      // The slot was read and written through the generic proxy; order that
-      // before the bulk copy that will refill it.
+      // This warp is done with the slot.  Its generic-proxy accesses are
+      // ordered before the bulk copy that refills it; the last warp to finish
+      // issues that copy (tile i + kStages) at once.
       fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        if (atomicAdd(&s.done[st], 1) == kWarps - 1) {
+          s.done[st] = 0;
+          __threadfence_block();
+          const int nx = i + kStages;
+          if (nx < count) {
+            uint8_t *slot = smem + st * slot_bytes;
+            issue_record<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[nx]);
+            issue_rest<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[nx], s.tl_n[nx],
+                                     s.tl_coord[nx]);
+          }
+        }
+      }
+      __syncwarp();
     } else {
       if (!mbar_wait_bounded(&s.bar[st], parity)) s.abort = 1;
       __syncthreads();
@@ -1416,7 +1444,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
   }
   if (i < count) {
     // A copy did not complete in time: flag it, then give the copies still in
-    // flight into this CTA's shared memory a bounded chance to land.
+    // flight into this CTA's shared memory a bounded chance to land.  On the
+    // GDN-bf16 path every tile before i had all its warps finish, so its
+    // slot's refill (tile + kStages) has been issued.
+    if constexpr (TR::kTok == 2) issued = (i + kStages < count) ? i + kStages : count;
     if (tid == 0) {
       atomicOr(p.err, kErrTimeout);
       for (int k = i; k < issued; ++k)
@@ -1625,7 +1656,21 @@ cudaError_t decode_t(const KParams &p, cudaStream_t st) {
   if (grid > tiles) grid = tiles;
   const int need = (tiles + kMaxTilesPerCta - 1) / kMaxTilesPerCta;
   if (grid < need) grid = need;
-  decode_kernel<D, BF16, KDA><<<grid, kThreads, smem, st>>>(p);
+  // programmatic dependent launch: the kernel waits (griddepcontrol.wait)
+  // before its first global access, so its launch and shared-memory setup
+  // may overlap the tail of the previous kernel in the stream
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<D, BF16, KDA>, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
