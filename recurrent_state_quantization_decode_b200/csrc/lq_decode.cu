@@ -890,13 +890,76 @@ __device__ __forceinline__ void digit_scales(float M, float &up, float &down) {
   }
 }
 
+// Window gate of a GDN tile, Gamma_t = alpha_1 ... alpha_t: the n buffered
+// gates (a 16-float line in shared memory) and the current one, multiplied
+// left to right in registers (every lane the same value).
+__device__ __forceinline__ float gate_product(const float *sbg, float alpha0, int n) {
+  const float4 *g4 = reinterpret_cast<const float4 *>(sbg);
+  float g[kGdnGateStride];
+#pragma unroll
+  for (int u = 0; u < kGdnGateStride / 4; ++u) {
+    const float4 v = g4[u];
+    g[4 * u] = v.x;
+    g[4 * u + 1] = v.y;
+    g[4 * u + 2] = v.z;
+    g[4 * u + 3] = v.w;
+  }
+  float P = 1.0f;
+#pragma unroll
+  for (int s = 0; s < kGdnGateStride; ++s) {
+    const float a = (s < n) ? g[s] : (s == n ? alpha0 : 1.0f);
+    P *= a;
+  }
+  return P;
+}
+
+// GDN with bf16 inputs: the row-compensator lines' dot products with
+// Gamma o q and Gamma o k over all D key channels, for the lines c = first,
+// first + stride, ... (lane l takes channels l, l + 32, ...).  Writes
+// cpart[c][0] (q, k); column lines are skipped.
+template <int D, class TK>
+__device__ __forceinline__ void comp_dots_fast(TK &x, const __nv_bfloat16 *sq,
+                                               const __nv_bfloat16 *sk, const float *sbg,
+                                               const float *rcv, const int *rcid, float alpha0,
+                                               int n, int K, int first, int stride) {
+  const int lane = threadIdx.x & 31;
+  constexpr int CPL = (D + 31) / 32;
+  float gq[CPL], gk[CPL];
+  const float Gm = gate_product(sbg, alpha0, n);
+#pragma unroll
+  for (int u = 0; u < CPL; ++u) {
+    const int j = lane + 32 * u;
+    gq[u] = j < D ? Gm * __bfloat162float(sq[j]) : 0.0f;
+    gk[u] = j < D ? Gm * __bfloat162float(sk[j]) : 0.0f;
+  }
+  for (int c = first; c < K; c += stride) {
+    if (rcid[c] >= D) continue;
+    float dq = 0.0f, dk = 0.0f;
+#pragma unroll
+    for (int u = 0; u < CPL; ++u) {
+      const int j = lane + 32 * u;
+      const float cv = j < D ? rcv[c * D + j] : 0.0f;
+      dq = fmaf(cv, gq[u], dq);
+      dk = fmaf(cv, gk[u], dk);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      dq += __shfl_xor_sync(kFull, dq, o);
+      dk += __shfl_xor_sync(kFull, dk, o);
+    }
+    if (lane == 0) {
+      x.cpart[c][0][0] = dq;
+      x.cpart[c][0][1] = dk;
+    }
+  }
+}
+
 // GDN with bf16 inputs: warp c < 2 * NSPAN does the per-channel work of int8
 // MMA k-chunk c, the 32 columns 64h + 16t + 8u + e (h = c / 2, u = c % 2,
 // t < 4, e < 8) that the chunk's codes cover; lane l takes t = l / 8, e = l % 8.
 // Each chunk's digits get their own power-of-two scale, so the max is a warp
-// reduction.  Writes q, k, v (fp32), Gamma, m o Gamma, the chunk's digits and
-// scales and its partial row-compensator dots (cpart[line][c]); warp 0 also
-// appends k_t.
+// reduction.  Writes q, k, v (fp32), Gamma, m o Gamma and the chunk's digits
+// and scales; warp 0 also appends k_t.
 template <int D, class TK>
 __device__ __forceinline__ void channel_chunk_fast(const KParams &p, TK &x,
                                                    const __nv_bfloat16 *sq,
@@ -909,11 +972,7 @@ __device__ __forceinline__ void channel_chunk_fast(const KParams &p, TK &x,
   const int tq = lane >> 3;
   const int j = 64 * (c >> 1) + 16 * tq + 8 * (c & 1) + (lane & 7);
   const bool valid = D >= 64 || tq < 2;
-  // window gate Gamma_t = prod of the n buffered gates and the current one
-  float P = (lane < n) ? sbg[lane] : (lane == n ? alpha0 : 1.0f);
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) P *= __shfl_xor_sync(kFull, P, o);
-  const float Gm = P;
+  const float Gm = gate_product(sbg, alpha0, n);
   float q = 0.0f, k = 0.0f, xq = 0.0f, xk = 0.0f;
   if (valid) {
     q = __bfloat162float(sq[j]);
@@ -945,21 +1004,6 @@ __device__ __forceinline__ void channel_chunk_fast(const KParams &p, TK &x,
   if (lane == 0) {
     x.xscale[0][c] = dnq;
     x.xscale[1][c] = dnk;
-  }
-  // row-compensator lines dotted with Gamma o q and Gamma o k over this chunk
-  const float gq = Gm * q, gk = Gm * k;
-  for (int c0 = 0; c0 < p.K; c0 += 4) {
-    float v[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int line = c0 + i;
-      const float cvj = (valid && line < p.K && rcid[line] < D) ? rcv[line * D + j] : 0.0f;
-      v[2 * i] = cvj * gq;
-      v[2 * i + 1] = cvj * gk;
-    }
-    const float tot = warp_sum8(v, lane);
-    const int vi = (lane >> 2) & 7, line = c0 + (vi >> 1);
-    if ((lane & 3) == 0 && line < p.K) x.cpart[line][c][vi & 1] = tot;
   }
 }
 
@@ -1003,11 +1047,11 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
   // ---- Phases A and B ----
   constexpr bool kFast = DecodeTraits<D, BF16, KDA>::kFast;
   constexpr int NCH = 2 * G::NSPAN;    // int8 MMA k-chunks (GDN-bf16: one channel warp each)
-  constexpr int CWP = kFast ? NCH : CW;  // warps holding compensator partial dots
+  constexpr int CWP = kFast ? 1 : CW;  // warps holding compensator partial dots
   uint4 A[2][G::NSPAN];
   if constexpr (kFast) {
-    // one warp per k-chunk for the channels, one for the buffer coefficients;
-    // the other row warps fetch their code fragments
+    // one warp per k-chunk for the channels, one for the buffer coefficients,
+    // the others for the row-compensator dot products
     if (warp < NCH) {
       if (warp < G::NRB) load_codes<D>(codes, A);
       channel_chunk_fast<D>(p, x, reinterpret_cast<const __nv_bfloat16 *>(sq),
@@ -1021,8 +1065,13 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
       coef_mma<D>(x, reinterpret_cast<const __nv_bfloat16 *>(sbk),
                   reinterpret_cast<const __nv_bfloat16 *>(sk),
                   reinterpret_cast<const __nv_bfloat16 *>(sq), sbg, alpha0, n);
-    } else if (warp < G::NRB) {
-      load_codes<D>(codes, A);
+    } else {
+      // the remaining warps fetch their code fragments, then share out the
+      // row-compensator lines' dot products
+      if (warp < G::NRB) load_codes<D>(codes, A);
+      comp_dots_fast<D>(x, reinterpret_cast<const __nv_bfloat16 *>(sq),
+                        reinterpret_cast<const __nv_bfloat16 *>(sk), sbg, rcv, rcid, alpha0, n,
+                        p.K, warp - NCH - 1, kWarps - NCH - 1);
     }
     // the one CTA barrier of a plain token: the copies of this tile have
     // landed for every thread, and the previous tile's slot is free
