@@ -1,7 +1,7 @@
 """Benchmark of the int8-state LeapQuant GDN/KDA decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload qwen35_9b_gdn|kimi_linear_kda] [--layers L]
+                    [--workload qwen35_9b_gdn|kimi_linear_kda|gdn_sweep_bB] [--layers L]
 
 One step = one 16-token quantization window (15 plain decode tokens and the
 boundary token whose kernel also folds, compensates, smooths and requantizes)
@@ -47,7 +47,8 @@ METRIC = ("decode tokens/s·head (int8 state) & achieved HBM GB/s vs 8 TB/s; "
           "speedup vs fp32 state")
 UNIT = "tile-steps/s"
 NOMINAL_HBM_GBS = 8000.0
-WORKLOADS = {"qwen35_9b_gdn": wl.QWEN35_9B_GDN, "kimi_linear_kda": wl.KIMI_LINEAR_KDA}
+WORKLOADS = {"qwen35_9b_gdn": wl.QWEN35_9B_GDN, "kimi_linear_kda": wl.KIMI_LINEAR_KDA,
+             **{f"gdn_sweep_b{b}": wl.sweep_workload(b) for b in wl.SWEEP_BATCHES}}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_qwen35_9b_gdn.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "recurrent_state_quantization_decode_b200", "csrc", f)
                   for f in ("lq_decode.cu", "lq_internal.h")]

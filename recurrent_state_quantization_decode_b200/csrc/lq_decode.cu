@@ -550,18 +550,21 @@ __device__ void quantize_tile(SC &s, double *colpart, float *colmax,
       double e0 = 0.0, e1 = 0.0;
 #pragma unroll
       for (int h = 0; h < G::NSPAN; ++h) {
-        double cp[16];
+        // eight columns at a time keeps the fp64 partials in few registers;
+        // lane g ends with column 8 hh + g of the batch
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const double a = SX(0, h, e), b = SX(1, h, e);
-          e0 = fma(a, a, e0);
-          e1 = fma(b, b, e1);
-          cp[e] = fma(a, a, b * b);
+        for (int hh = 0; hh < 2; ++hh) {
+          double cp[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const double a = SX(0, h, 8 * hh + e), b = SX(1, h, 8 * hh + e);
+            e0 = fma(a, a, e0);
+            e1 = fma(b, b, e1);
+            cp[e] = fma(a, a, b * b);
+          }
+          butterfly_g<8>(cp, lane, AddOp());
+          if (chunk_valid<D>(t)) colpart[warp * D + frag_col(h, t, 8 * hh + g)] = cp[0];
         }
-        butterfly_g<16>(cp, lane, AddOp());
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-          if (chunk_valid<D>(t)) colpart[warp * D + frag_col(h, t, 2 * g + u)] = cp[u];
       }
       e0 += __shfl_xor_sync(kFull, e0, 1);
       e0 += __shfl_xor_sync(kFull, e0, 2);
@@ -680,13 +683,15 @@ __device__ void quantize_tile(SC &s, double *colpart, float *colmax,
   if (rows_here) {
 #pragma unroll
     for (int h = 0; h < G::NSPAN; ++h) {
-      float cm[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) cm[e] = fmaxf(fabsf(SX(0, h, e)), fabsf(SX(1, h, e)));
-      butterfly_g<16>(cm, lane, MaxOp());
+      for (int hh = 0; hh < 2; ++hh) {
+        float cm[8];
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
-        if (chunk_valid<D>(t)) colmax[warp * D + frag_col(h, t, 2 * g + u)] = cm[u];
+        for (int e = 0; e < 8; ++e)
+          cm[e] = fmaxf(fabsf(SX(0, h, 8 * hh + e)), fabsf(SX(1, h, 8 * hh + e)));
+        butterfly_g<8>(cm, lane, MaxOp());
+        if (chunk_valid<D>(t)) colmax[warp * D + frag_col(h, t, 8 * hh + g)] = cm[0];
+      }
     }
   }
   __syncthreads();
