@@ -135,7 +135,20 @@ struct DecodeTraits {
   static constexpr bool kKtOverCodes = kFast && kMaxWindow * FG<D>::PADW * 4 <= D * D;
   static constexpr int kStages = kFast ? 3 : 2;
   static constexpr int kTok = kFast ? 2 : 1;  // per-token scratch buffers
+  // the fold's rank-W update on the tf32 tensor path (3 products per term)
+  static constexpr bool kMmaFold = kFast && D >= 64;
 };
+
+// Scaled-key layout of the tensor-path fold update: row s of width D + 8 (the
+// 8-float pad puts the four k rows a warp reads at once in different banks);
+// column c sits where lane g of n8 tile j of span h reads it, c = 64h +
+// 16(g/2) + 2j + g%2, so that the accumulators land in the state's layout.
+template <int D>
+__host__ __device__ constexpr int kt_mma_stride() { return D + 8; }
+__device__ __forceinline__ int kt_mma_pos(int c) {
+  const int r = c & 63;
+  return (c & ~63) + 8 * ((r & 15) >> 1) + 2 * (r >> 4) + (r & 1);
+}
 
 // The scaled-key array lives in the scratch unless the decode kernel keeps it
 // over the staged codes (GDN with bf16 inputs).
@@ -311,6 +324,24 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D (16x8, fp32) += A (16x8, tf32, row) x B (8x8, tf32, col); c01 holds row g,
+// c23 row g + 8 (columns 2t, 2t + 1).
+__device__ __forceinline__ void mma_tf32(float2 &c01, float2 &c23, uint32_t a0, uint32_t a1,
+                                         uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c01.x), "+f"(c01.y), "+f"(c23.x), "+f"(c23.y)
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// x = hi + lo with hi, lo tf32 (round to nearest); hi * hi' + hi * lo' + lo * hi'
+// then reproduces an fp32 product to about 2^-22 relative.
+__device__ __forceinline__ void tf32_split(float x, uint32_t &hi, uint32_t &lo) {
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(x - __uint_as_float(hi)));
+}
+
 // Exact split of x into four radix-128 digits with the power-of-two scale
 // s = 2^(E-6), where max|x| = M < 2^E:  x = s (d0 + d1/128 + d2/128^2 +
 // d3/128^3) + r with |r| <= s / (2 * 128^3).  Every step is exact in fp32,
@@ -430,7 +461,7 @@ __device__ __forceinline__ void load_codes(const uint8_t *codes, uint4 (&A)[2][F
 //          + Gamma_j * (compensator lines),
 // with kt_s = k_s o (decay ratio to the last token) in kt (rows of PADW) and m o Gamma in
 // x.mG.  rsig, rcv, rcid point at the staged record; bd at the staged deltas.
-template <int D, class SC>
+template <int D, bool MMA = false, class SC>
 __device__ __forceinline__ void build_state(const SC &x, const float *kt,
                                             const uint4 (&A)[2][FG<D>::NSPAN],
                                             const float *rsig, const float *rcv, const int *rcid,
@@ -464,8 +495,36 @@ __device__ __forceinline__ void build_state(const SC &x, const float *kt,
       for (int e2 = 0; e2 < 8; ++e2) S[0][h][e2] = S[1][h][e2] = make_float2(0.0f, 0.0f);
     }
   }
+  if constexpr (MMA) {
+    // rank-nent update on the tf32 tensor path: A = d (16 rows x 8 tokens),
+    // B = scaled keys (8 tokens x 8 columns) in the layout of kt_mma_pos;
+    // tokens at or beyond nent contribute zero
+    constexpr int P = kt_mma_stride<D>();
+#pragma unroll
+    for (int ks = 0; ks < kMaxWindow / 8; ++ks) {
+      if (8 * ks >= nent) break;
+      const int s0 = 8 * ks + t, s1 = s0 + 4;
+      uint32_t ah[4], al[4];
+      tf32_split(s0 < nent ? bd[s0 * D + r0] : 0.0f, ah[0], al[0]);
+      tf32_split(s0 < nent ? bd[s0 * D + r1] : 0.0f, ah[1], al[1]);
+      tf32_split(s1 < nent ? bd[s1 * D + r0] : 0.0f, ah[2], al[2]);
+      tf32_split(s1 < nent ? bd[s1 * D + r1] : 0.0f, ah[3], al[3]);
+#pragma unroll
+      for (int h = 0; h < G::NSPAN; ++h)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int pos = 64 * h + 8 * j + g;
+          uint32_t bh0, bl0, bh1, bl1;
+          tf32_split(s0 < nent ? kt[s0 * P + pos] : 0.0f, bh0, bl0);
+          tf32_split(s1 < nent ? kt[s1 * P + pos] : 0.0f, bh1, bl1);
+          mma_tf32(S[0][h][j], S[1][h][j], al[0], al[1], al[2], al[3], bh0, bh1);
+          mma_tf32(S[0][h][j], S[1][h][j], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+          mma_tf32(S[0][h][j], S[1][h][j], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+        }
+    }
+  }
   // rank-nent update, two columns per packed FMA
-  for (int sl = 0; sl < nent; ++sl) {
+  for (int sl = 0; sl < (MMA ? 0 : nent); ++sl) {
     const float2 d0 = make_float2(bd[sl * D + r0], bd[sl * D + r0]);
     const float2 d1 = make_float2(bd[sl * D + r1], bd[sl * D + r1]);
 #pragma unroll
@@ -1329,16 +1388,26 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
       ktw = &s.kt[0][0];
     }
     if (tid < D) {
-      for (int sl = 0; sl < n; ++sl)
-        ktw[sl * G::PADW + padc(tid)] = to_f(sbk[sl * D + tid]) * x.rho[sl];
-      ktw[n * G::PADW + padc(tid)] = x.kf[tid];
+      if constexpr (DecodeTraits<D, BF16, KDA>::kMmaFold) {
+        constexpr int P = kt_mma_stride<D>();
+        const int pos = kt_mma_pos(tid);
+        for (int sl = 0; sl < n; ++sl)
+          ktw[sl * P + pos] = to_f(sbk[sl * D + tid]) * x.rho[sl];
+        ktw[n * P + pos] = x.kf[tid];
+      } else {
+        for (int sl = 0; sl < n; ++sl)
+          ktw[sl * G::PADW + padc(tid)] = to_f(sbk[sl * D + tid]) * x.rho[sl];
+        ktw[n * G::PADW + padc(tid)] = x.kf[tid];
+      }
     }
     __syncthreads();
     kt = ktw;
   } else {
     kt = &s.kt[0][0];
   }
-  if (warp < G::NRB) build_state<D>(x, kt, Af, rsig, rcv, rcid, sbd, n + 1, p.K, S);
+  if (warp < G::NRB)
+    build_state<D, DecodeTraits<D, BF16, KDA>::kMmaFold>(x, kt, Af, rsig, rcv, rcid, sbd, n + 1,
+                                                        p.K, S);
   __syncthreads();  // the staged codes and keys are now free for the quantizer's scratch
   quantize_tile<D>(s, reinterpret_cast<double *>(slot + L::QS_COLPART),
                    reinterpret_cast<float *>(slot + L::QS_COLMAX), S,
