@@ -136,7 +136,7 @@ struct DecodeTraits {
   static constexpr int kStages = kFast ? 3 : 2;
   static constexpr int kTok = kFast ? 2 : 1;  // per-token scratch buffers
   // the fold's rank-W update on the tf32 tensor path (3 products per term)
-  static constexpr bool kMmaFold = kFast && D >= 64;
+  static constexpr bool kMmaFold = D >= 64;
 };
 
 // Scaled-key layout of the tensor-path fold update: row s of width D + 8 (the
@@ -145,6 +145,15 @@ struct DecodeTraits {
 // 16(g/2) + 2j + g%2, so that the accumulators land in the state's layout.
 template <int D>
 __host__ __device__ constexpr int kt_mma_stride() { return D + 8; }
+__device__ __forceinline__ int kt_mma_pos(int c);
+// Index of scaled key (token s, column c) in the fold's key array.
+template <int D, bool MMA>
+__device__ __forceinline__ int kt_index(int s, int c) {
+  if constexpr (MMA)
+    return s * kt_mma_stride<D>() + kt_mma_pos(c);
+  else
+    return s * FG<D>::PADW + padc(c);
+}
 __device__ __forceinline__ int kt_mma_pos(int c) {
   const int r = c & 63;
   return (c & ~63) + 8 * ((r & 15) >> 1) + 2 * (r >> 4) + (r & 1);
@@ -1110,6 +1119,7 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
 
   // ---- Phases A and B ----
   constexpr bool kFast = DecodeTraits<D, BF16, KDA>::kFast;
+  constexpr bool kMmaF = DecodeTraits<D, BF16, KDA>::kMmaFold;
   constexpr int NCH = 2 * G::NSPAN;    // int8 MMA k-chunks (GDN-bf16: one channel warp each)
   constexpr int CWP = kFast ? 1 : CW;  // warps holding compensator partial dots
   uint4 A[2][G::NSPAN];
@@ -1163,10 +1173,10 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
       // the current token backwards, applied to the buffered keys
       acc = KDA ? sa[j] : alpha0;
       for (int sl = n - 1; sl >= 0; --sl) {
-        s.kt[sl][padc(j)] = to_f(sbk[sl * D + j]) * acc;
+        (&s.kt[0][0])[kt_index<D, kMmaF>(sl, j)] = to_f(sbk[sl * D + j]) * acc;
         acc *= KDA ? sbg[sl * D + j] : sbg[sl];
       }
-      s.kt[n][padc(j)] = kj;
+      (&s.kt[0][0])[kt_index<D, kMmaF>(n, j)] = kj;
     }
     x.G[j] = acc;
     const float mj = rm[j];
@@ -1230,7 +1240,7 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
     for (int sl = warp - CW; sl <= n; sl += kWarps - CW) {
       float c = 0.0f, a = 0.0f;
       for (int j = lane; j < D; j += 32) {
-        const float kv = s.kt[sl][padc(j)];
+        const float kv = (&s.kt[0][0])[kt_index<D, kMmaF>(sl, j)];
         c = fmaf(kv, x.kf[j], c);
         a = fmaf(kv, x.qf[j], a);
       }
