@@ -199,6 +199,21 @@ lq_status lq_decode_step_host_noalloc(const lq_config *cfg, const void *q_host,
                                       const lq_state *st, void *out_host, const int32_t *active,
                                       void *stream);
 
+/* TESTING ONLY (no counterpart on the pages): the failure path of the
+ * bounded waits.  Runs lq_decode_step except that the first CTA issues no
+ * copies for its first ring slot, so that its wait on that slot expires
+ * after `wait_limit` polls (> 0; production launches use 2^24).  That CTA
+ * sets the timeout bit of the error word, waits (bounded) for its other
+ * copies, and returns without touching the rest of its tiles; nothing is in
+ * flight into the withheld slot.  Returns the launch status; afterwards
+ * lq_get_last_error reports LQ_ERR_TIMEOUT.  The state of the skipped tiles
+ * is left inconsistent: re-initialise it before further use.  Inputs as for
+ * lq_decode_step (all sequences active). */
+lq_status lq_test_decode_step_timeout(const lq_config *cfg, const void *q, const void *k,
+                                      const void *v, const float *alpha, const float *beta,
+                                      const lq_state *st, void *out, uint32_t wait_limit,
+                                      void *stream);
+
 /* Fold a partially filled window now (0 < buf_n < W) for the selected
  * sequences, exactly as the boundary fold does (news article, paragraph 3:
  * reconstruct and quantize at the boundary).  Used at the end of a sequence

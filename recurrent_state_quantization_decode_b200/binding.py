@@ -33,7 +33,8 @@ LQ_DTYPE_F32, LQ_DTYPE_BF16 = 0, 1
 EXPORTED = ("lq_version", "lq_status_string", "lq_state_layout", "lq_state_bytes",
             "lq_state_init", "lq_decode_step", "lq_decode_step_host",
             "lq_decode_step_host_noalloc", "lq_window_flush",
-            "lq_fp32_decode_step", "lq_state_dequantize", "lq_get_last_error")
+            "lq_fp32_decode_step", "lq_state_dequantize", "lq_get_last_error",
+            "lq_test_decode_step_timeout")
 
 
 class lq_config(ctypes.Structure):
@@ -74,6 +75,8 @@ _sig = {
     "lq_fp32_decode_step": ([_CFG, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "lq_state_dequantize": ([_CFG, _ST, ctypes.c_int32, _P, _P], ctypes.c_int),
     "lq_get_last_error": ([_ST, _P], ctypes.c_int),
+    "lq_test_decode_step_timeout": ([_CFG, _P, _P, _P, _P, _P, _ST, _P, ctypes.c_uint32, _P],
+                                    ctypes.c_int),
 }
 for _name, (_args, _res) in _sig.items():
     _f = getattr(_lib, _name)
@@ -169,6 +172,17 @@ def lq_decode_step(cfg, q, k, v, alpha, beta, state: lq_state, out, active=None,
     _check(_lib.lq_decode_step(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
                                _ptr(beta), ctypes.byref(state), _ptr(out), _ptr(active),
                                _stream(stream)), "lq_decode_step")
+
+
+def lq_test_decode_step_timeout(cfg, q, k, v, alpha, beta, state: lq_state, out,
+                                wait_limit: int, stream=None) -> None:
+    """Testing only: lq_decode_step in which the first CTA withholds the copies
+    of its first ring slot, so that its bounded wait (wait_limit polls) expires
+    and the error word reports LQ_ERR_TIMEOUT."""
+    _check(_lib.lq_test_decode_step_timeout(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(alpha), _ptr(beta), ctypes.byref(state),
+                                            _ptr(out), ctypes.c_uint32(wait_limit),
+                                            _stream(stream)), "lq_test_decode_step_timeout")
 
 
 def lq_decode_step_host(cfg, q_host, k_host, v_host, alpha_host, beta_host, state: lq_state,

@@ -77,6 +77,7 @@ KParams make_params(const lq_config *c, const lq_state *st) {
   p.out_bf16 = c->out_dtype == LQ_DTYPE_BF16;
   p.smooth = c->smooth == 0.0f ? 0 : (c->smooth == 0.5f ? 1 : 2);
   p.L = lq::record_layout(c->d, c->n_comp);
+  p.wait_limit = lq::kWaitLimitDefault;
   if (st != nullptr) {
     p.records = static_cast<uint8_t *>(st->records);
     p.buf_k = st->buf_k;
@@ -177,6 +178,27 @@ lq_status lq_decode_step(const lq_config *cfg, const void *q, const void *k, con
   p.beta = beta;
   p.out = out;
   p.mask = active;
+  return from_cuda(lq::launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
+lq_status lq_test_decode_step_timeout(const lq_config *cfg, const void *q, const void *k,
+                                      const void *v, const float *alpha, const float *beta,
+                                      const lq_state *st, void *out, uint32_t wait_limit,
+                                      void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if ((s = check_io(cfg, q, k, v, alpha, beta, out)) != LQ_OK) return s;
+  if (cfg->batch == 0 || wait_limit == 0) return LQ_ERR_INVALID_ARG;
+  KParams p = make_params(cfg, st);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.out = out;
+  p.wait_limit = wait_limit;
+  p.withhold = 1;
   return from_cuda(lq::launch_decode(p, static_cast<cudaStream_t>(stream)));
 }
 

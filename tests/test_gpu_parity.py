@@ -394,6 +394,47 @@ def test_corrupt_phase_sets_error_word_and_skips_tile():
     assert P.normwise(o[0].astype(np.float64), ref) <= P.REL_TOL
 
 
+@pytest.mark.parametrize("bf16,gate", [(True, wl.GATE_SCALAR), (True, wl.GATE_DIAG)])
+def test_bounded_wait_expiry_reports_timeout(bf16, gate):
+    """The first CTA withholds its first slot's copies: its wait expires after a
+    few polls, the error word says LQ_ERR_TIMEOUT, its tiles are left alone,
+    every other CTA's tiles match a normal step, and the context stays usable."""
+    w = wl.Workload("t", 64, 16, 32, 128, gate, bf16, 1)
+    rng = np.random.default_rng(9)
+    S0, _, _ = wl.initial_states(rng, w.tiles, w.d, w.d)
+    ti = wl.token_inputs(rng, w, 1)
+    cfg = B.config_for(w)
+    S0_dev = torch.from_numpy(S0).cuda()
+    dev = P.DeviceInputs(ti, bf16)
+    outs = []
+    for faulted in (False, True):
+        ds = B.DeviceState(cfg)
+        B.lq_state_init(cfg, S0_dev, ds.st)
+        out = torch.full((w.batch, w.num_v_heads, w.d), float("nan"), device="cuda")
+        if faulted:
+            B.lq_test_decode_step_timeout(cfg, *dev.token(0), ds.st, out, wait_limit=2000)
+            assert B.lq_get_last_error(ds.st) == B.LQ_ERR_TIMEOUT
+        else:
+            B.lq_decode_step(cfg, *dev.token(0), ds.st, out)
+            assert B.lq_get_last_error(ds.st) == B.LQ_OK
+        outs.append(out.reshape(w.tiles, w.d).cpu().numpy())
+    normal, faulted = outs
+    assert np.all(np.isnan(faulted[0]))              # the first CTA's first tile: untouched
+    done = ~np.isnan(faulted).any(axis=1)
+    skipped = np.flatnonzero(~done)                   # the first CTA's tiles: 0, g, 2g, ...
+    assert skipped[0] == 0 and len(skipped) < w.tiles // 100
+    if len(skipped) > 1:
+        assert np.array_equal(skipped, skipped[1] * np.arange(len(skipped)))
+    assert np.array_equal(faulted[done], normal[done])
+    # the context is still usable: a normal step on a fresh state succeeds
+    ds = B.DeviceState(cfg)
+    B.lq_state_init(cfg, S0_dev, ds.st)
+    out = torch.empty((w.batch, w.num_v_heads, w.d), device="cuda")
+    B.lq_decode_step(cfg, *dev.token(0), ds.st, out)
+    assert B.lq_get_last_error(ds.st) == B.LQ_OK
+    assert torch.isfinite(out).all()
+
+
 def test_host_entry_point_matches_device_entry_point():
     w = wl.Workload("h", 4, 2, 4, 128, wl.GATE_SCALAR, True, 20)
     rng = np.random.default_rng(6)
