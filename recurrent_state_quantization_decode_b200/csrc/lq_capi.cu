@@ -226,12 +226,11 @@ lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const vo
   uint8_t *da = dv + round256(nv);
   uint8_t *db = da + round256(na);
   uint8_t *dout = db + round256(nb);
-  cudaError_t e;
-  if ((e = cudaMemcpyAsync(dq, q_host, nq, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(dk, k_host, nq, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(dv, v_host, nv, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(da, alpha_host, na, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(db, beta_host, nb, cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+  if (cudaMemcpyAsync(dq, q_host, nq, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k_host, nq, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v_host, nv, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(da, alpha_host, na, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(db, beta_host, nb, cudaMemcpyHostToDevice, cs) != cudaSuccess)
     return LQ_ERR_CUDA;
   KParams p = make_params(cfg, st);
   p.q = dq;
@@ -241,8 +240,8 @@ lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const vo
   p.beta = reinterpret_cast<const float *>(db);
   p.out = dout;
   p.mask = active;
-  if ((e = lq::launch_decode(p, cs)) != cudaSuccess) return LQ_ERR_CUDA;
-  if ((e = cudaMemcpyAsync(out_host, dout, no, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+  if (lq::launch_decode(p, cs) != cudaSuccess) return LQ_ERR_CUDA;
+  if (cudaMemcpyAsync(out_host, dout, no, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
     return LQ_ERR_CUDA;
   return LQ_OK;
 }

@@ -223,17 +223,6 @@ __device__ __forceinline__ void st_out(void *p, size_t i, float x, int bf16) {
     reinterpret_cast<float *>(p)[i] = x;
 }
 
-__device__ __forceinline__ void load16(const float *src, float (&dst)[16]) {
-  const float4 *s4 = reinterpret_cast<const float4 *>(src);
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const float4 v = s4[u];
-    dst[4 * u] = v.x;
-    dst[4 * u + 1] = v.y;
-    dst[4 * u + 2] = v.z;
-    dst[4 * u + 3] = v.w;
-  }
-}
 
 // int8 code e (0..15) of a 16-byte chunk as a float, without an int->float
 // conversion: the byte, biased to unsigned, becomes the low mantissa byte of
@@ -262,12 +251,9 @@ __device__ __forceinline__ void fence_mbar_init() {
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long *bar, uint32_t bytes) {
-  unsigned long long state;
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 %0, [%1], %2;"
-               : "=l"(state)
-               : "r"(smem_u32(bar)), "r"(bytes)
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
                : "memory");
-  (void)state;
 }
 
 __device__ __forceinline__ void mbar_expect_tx(unsigned long long *bar, uint32_t bytes) {
@@ -1278,16 +1264,16 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
         mma_s8(acc[2 * hh], A[0][hh].x, A[1][hh].x, A[0][hh].y, A[1][hh].y, Bw.x, Bw.y);
         mma_s8(acc[2 * hh + 1], A[0][hh].z, A[1][hh].z, A[0][hh].w, A[1][hh].w, Bw.z, Bw.w);
       }
-      const float pair = (t & 1) ? 1.0f / 16384.0f : 1.0f;
+      // digits 2t, 2t+1 combine exactly as one integer (|.| < 2^26) before
+      // the chunk scale applies
+      const float pair = (t & 1) ? 1.0f / (128.0f * 16384.0f) : 1.0f / 128.0f;
       p0 = 0.0f;
       p1 = 0.0f;
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
         const float sc = x.xscale[t >> 1][c] * pair;
-        p0 = fmaf(sc, static_cast<float>(acc[c][0]) +
-                          static_cast<float>(acc[c][1]) * (1.0f / 128.0f), p0);
-        p1 = fmaf(sc, static_cast<float>(acc[c][2]) +
-                          static_cast<float>(acc[c][3]) * (1.0f / 128.0f), p1);
+        p0 = fmaf(sc, static_cast<float>(acc[c][0] * 128 + acc[c][1]), p0);
+        p1 = fmaf(sc, static_cast<float>(acc[c][2] * 128 + acc[c][3]), p1);
       }
       sq0 = 1.0f;
       sk0 = 1.0f;
