@@ -765,8 +765,22 @@ __device__ void quantize_tile(SC &s, double *colpart, float *colmax,
   }
   __syncthreads();
 
-  // Per-row scales and int8 codes.
+  // Per-row scales and int8 codes.  1/m is loaded once for both rows.
   if (rows_here) {
+#pragma unroll
+    for (int h = 0; h < G::NSPAN; ++h) {
+      if (!chunk_valid<D>(t)) continue;
+      const float4 *im4 = reinterpret_cast<const float4 *>(&s.invm[padc(frag_col(h, t, 0))]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 im = im4[u];
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          S[rr][h][2 * u] = __fmul2_rn(S[rr][h][2 * u], make_float2(im.x, im.y));
+          S[rr][h][2 * u + 1] = __fmul2_rn(S[rr][h][2 * u + 1], make_float2(im.z, im.w));
+        }
+      }
+    }
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int row = rr ? r1 : r0;
@@ -774,16 +788,9 @@ __device__ void quantize_tile(SC &s, double *colpart, float *colmax,
 #pragma unroll
       for (int h = 0; h < G::NSPAN; ++h) {
         if (!chunk_valid<D>(t)) continue;
-        const float4 *im4 = reinterpret_cast<const float4 *>(&s.invm[padc(frag_col(h, t, 0))]);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 im = im4[u];
-          S[rr][h][2 * u] = __fmul2_rn(S[rr][h][2 * u], make_float2(im.x, im.y));
-          S[rr][h][2 * u + 1] = __fmul2_rn(S[rr][h][2 * u + 1], make_float2(im.z, im.w));
-          bmax = fmaxf(bmax, fmaxf(fmaxf(fabsf(S[rr][h][2 * u].x), fabsf(S[rr][h][2 * u].y)),
-                                   fmaxf(fabsf(S[rr][h][2 * u + 1].x),
-                                         fabsf(S[rr][h][2 * u + 1].y))));
-        }
+        for (int e2 = 0; e2 < 8; ++e2)
+          bmax = fmaxf(bmax, fmaxf(fabsf(S[rr][h][e2].x), fabsf(S[rr][h][e2].y)));
       }
       bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, 1));
       bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, 2));
@@ -803,13 +810,12 @@ __device__ void quantize_tile(SC &s, double *colpart, float *colmax,
         uint32_t w[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          // |x| <= 127 (1 + 2^-23) by construction; the clamp guards the bound
+          // |x| <= 127 (1 + 2^-23) since bmax is the row's max, so x rounds
+          // into [-127, 127] without a clamp
           const float2 xa = __fmul2_rn(S[rr][h][2 * u], inv2);
           const float2 xb = __fmul2_rn(S[rr][h][2 * u + 1], inv2);
-          const float x0 = fminf(fmaxf(xa.x, -127.0f), 127.0f) + kRoundMagic;
-          const float x1 = fminf(fmaxf(xa.y, -127.0f), 127.0f) + kRoundMagic;
-          const float x2 = fminf(fmaxf(xb.x, -127.0f), 127.0f) + kRoundMagic;
-          const float x3 = fminf(fmaxf(xb.y, -127.0f), 127.0f) + kRoundMagic;
+          const float x0 = xa.x + kRoundMagic, x1 = xa.y + kRoundMagic;
+          const float x2 = xb.x + kRoundMagic, x3 = xb.y + kRoundMagic;
           w[u] = __byte_perm(__byte_perm(__float_as_uint(x0), __float_as_uint(x1), 0x0040u),
                              __byte_perm(__float_as_uint(x2), __float_as_uint(x3), 0x0040u),
                              0x5410u);
