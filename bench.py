@@ -351,6 +351,51 @@ def whole_job_rate(units_per_step: int, world: int, steps: int, ms_max: float) -
     return world * units_per_step * steps / (ms_max / 1e3)
 
 
+PREFILL_TOKENS = 256
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # SMs x fp32 lanes x 2 flops x max clock
+
+
+def prefill_measure(B, w: wl.Workload, ly, stream, device, world: int) -> dict:
+    """lq_prefill of one layer's tiles over a PREFILL_TOKENS-token prompt
+    (seeded inputs), CUDA-event timed after one warm-up run.  Flops count the
+    exact recurrence's 7 d^2 per tile-token (decay, S k, update, S q)."""
+    import torch
+
+    T = PREFILL_TOKENS
+    ti = wl.token_inputs(np.random.default_rng(4242), w, T)
+    dt = torch.bfloat16 if w.io_bf16 else torch.float32
+    dev = {n: torch.from_numpy(getattr(ti, n)).to(device) for n in ("alpha", "beta")}
+    for n in ("q", "k", "v"):
+        dev[n] = torch.from_numpy(getattr(ti, n)).to(device=device, dtype=dt)
+    out = torch.empty((T, w.batch, w.num_v_heads, w.d), dtype=torch.float32, device=device)
+    ds = B.DeviceState(ly.cfg, device=device)
+    runs = 3
+
+    def run():
+        B.lq_prefill(ly.cfg, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], T,
+                     ly.S32, ds.st, out, stream=stream.cuda_stream)
+
+    with torch.cuda.stream(stream):
+        run()
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(runs):
+            run()
+        end.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(end) / runs, world, device)
+    tile_tokens = w.tiles * T
+    tflops = 7.0 * w.d * w.d * tile_tokens / (ms / 1e3) / 1e12
+    return {"tile_tokens_per_s": world * tile_tokens / (ms / 1e3), "ms": ms,
+            "prompt_tokens": T, "tiles": w.tiles,
+            "roofline": {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS,
+                         "unit": "TFLOP/s", "frac": tflops / FP32_ALU_TFLOPS,
+                         "peak_source": "148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"},
+            "kernel": "prefill_kernel (exact recurrence, state on chip, then quantizer)"}
+
+
 def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> None:
     import torch
     import torch.distributed as dist
@@ -493,6 +538,11 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "path": "lq_decode_step_host (pinned host q,k,v,alpha,beta in; o out)"}
 
+    # prefill of one layer's tiles over a prompt, ending in the quantizer
+    prefill = None
+    if not args.no_prefill:
+        prefill = prefill_measure(B, w, layers[0], stream, device, world)
+
     if rank != 0:
         return
     line = {
@@ -517,6 +567,8 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if prefill is not None:
+        line["prefill"] = prefill
     if world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
@@ -532,6 +584,7 @@ def main() -> None:
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

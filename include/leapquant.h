@@ -144,6 +144,25 @@ size_t lq_state_bytes(const lq_config *cfg, size_t *tile_bytes, size_t *buffer_b
 lq_status lq_state_init(const lq_config *cfg, const float *S0, const lq_state *st,
                         const int32_t *mask, void *stream);
 
+/* Prefill ending in the quantizer.  The pages describe the context being
+ * compressed into the fixed-size state that decode then reads and updates
+ * (AI Learning Platform article "LeapQuant: Efficient Linear Attention with
+ * Accurate Recurrent State Quantization", "Key Takeaway for Students"); this
+ * produces that state for a prompt.  Per tile, from S0 ([B][Hv][d][d] fp32,
+ * 16-byte aligned; NULL = zero states), it runs the exact recurrence in fp32
+ * for t = 0 .. T-1:
+ *   S <- S diag(alpha_t); S <- S + beta_t (v_t - S k_t) k_t^T; o_t = S q_t
+ * token by token with the state held on chip (not the chunked form), writes
+ * the T outputs (out: [T][B][Hv][d] in out_dtype; NULL = none), and then
+ * quantizes S_T into the record exactly as lq_state_init does (buffers empty,
+ * buf_n = 0).  Inputs are token-major: q, k [T][B][Hk][d], v [T][B][Hv][d]
+ * (in_dtype), alpha [T][B][Hv] (GDN) or [T][B][Hv][d] (KDA), beta
+ * [T][B][Hv], fp32.  T >= 0 (T = 0 quantizes S0).  mask: nullable [B] int32;
+ * masked-off sequences are left untouched. */
+lq_status lq_prefill(const lq_config *cfg, const void *q, const void *k, const void *v,
+                     const float *alpha, const float *beta, int32_t T, const float *S0,
+                     const lq_state *st, void *out, const int32_t *mask, void *stream);
+
 /* One decode token for every tile (zhichai.net summary, items 1-3; news
  * article paragraph 3).  Reads the int8 record as stored (no dequantized copy
  * in memory) and the buffered tokens, writes o_t = S_t q_t, appends

@@ -34,7 +34,7 @@ EXPORTED = ("lq_version", "lq_status_string", "lq_state_layout", "lq_state_bytes
             "lq_state_init", "lq_decode_step", "lq_decode_step_host",
             "lq_decode_step_host_noalloc", "lq_window_flush",
             "lq_fp32_decode_step", "lq_state_dequantize", "lq_get_last_error",
-            "lq_test_decode_step_timeout")
+            "lq_test_decode_step_timeout", "lq_prefill")
 
 
 class lq_config(ctypes.Structure):
@@ -77,6 +77,8 @@ _sig = {
     "lq_get_last_error": ([_ST, _P], ctypes.c_int),
     "lq_test_decode_step_timeout": ([_CFG, _P, _P, _P, _P, _P, _ST, _P, ctypes.c_uint32, _P],
                                     ctypes.c_int),
+    "lq_prefill": ([_CFG, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _ST, _P, _P, _P],
+                   ctypes.c_int),
 }
 for _name, (_args, _res) in _sig.items():
     _f = getattr(_lib, _name)
@@ -172,6 +174,15 @@ def lq_decode_step(cfg, q, k, v, alpha, beta, state: lq_state, out, active=None,
     _check(_lib.lq_decode_step(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
                                _ptr(beta), ctypes.byref(state), _ptr(out), _ptr(active),
                                _stream(stream)), "lq_decode_step")
+
+
+def lq_prefill(cfg, q, k, v, alpha, beta, T: int, S0, state: lq_state, out=None, mask=None,
+               stream=None) -> None:
+    """Exact recurrence over a T-token prompt (token-major inputs), outputs to
+    `out` ([T, B, Hv, d], optional), then the quantizer into `state`."""
+    _check(_lib.lq_prefill(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                           _ptr(beta), ctypes.c_int32(T), _ptr(S0), ctypes.byref(state),
+                           _ptr(out), _ptr(mask), _stream(stream)), "lq_prefill")
 
 
 def lq_test_decode_step_timeout(cfg, q, k, v, alpha, beta, state: lq_state, out,

@@ -181,6 +181,34 @@ lq_status lq_decode_step(const lq_config *cfg, const void *q, const void *k, con
   return from_cuda(lq::launch_decode(p, static_cast<cudaStream_t>(stream)));
 }
 
+lq_status lq_prefill(const lq_config *cfg, const void *q, const void *k, const void *v,
+                     const float *alpha, const float *beta, int32_t T, const float *S0,
+                     const lq_state *st, void *out, const int32_t *mask, void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if (T < 0) return LQ_ERR_INVALID_ARG;
+  if (T > 0 && (q == nullptr || k == nullptr || v == nullptr || alpha == nullptr ||
+                beta == nullptr))
+    return LQ_ERR_INVALID_ARG;
+  if (!aligned16(S0) || !aligned_to(alpha, 4) || !aligned_to(beta, 4) ||
+      !aligned_to(mask, 4) || !aligned_to(q, in_size(cfg)) || !aligned_to(k, in_size(cfg)) ||
+      !aligned_to(v, in_size(cfg)) || !aligned_to(out, out_size(cfg)))
+    return LQ_ERR_MISALIGNED;
+  if (cfg->batch == 0) return LQ_OK;
+  KParams p = make_params(cfg, st);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.T = T;
+  p.S_in = S0;
+  p.out = out;
+  p.mask = mask;
+  return from_cuda(lq::launch_prefill(p, static_cast<cudaStream_t>(stream)));
+}
+
 lq_status lq_test_decode_step_timeout(const lq_config *cfg, const void *q, const void *k,
                                       const void *v, const float *alpha, const float *beta,
                                       const lq_state *st, void *out, uint32_t wait_limit,

@@ -1729,6 +1729,147 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const KParams p) {
   if (tid == 0) p.buf_n[tile] = 0;
 }
 
+// Prefill: the exact recurrence over a prompt of T tokens with the tile's
+// fp32 state held in registers (the quantizer's fragment layout), then the
+// quantizer.  Per token: S <- S diag(alpha); y = S k; d = beta (v - y);
+// S <- S + d k^T; o = S q.  The next token's inputs are loaded while the
+// current one is computed.  One CTA per tile.
+template <int D, bool BF16, bool KDA>
+__global__ void __launch_bounds__(kThreads) prefill_kernel(const KParams p) {
+  using G = FG<D>;
+  using IT = in_t<BF16>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t *qscr = smem;  // D*D bytes of quantizer scratch
+  Scratch<D, false> &s = *reinterpret_cast<Scratch<D, false> *>(smem + D * D);
+  Tok<D> &x = s.tok[0];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int tile = blockIdx.x;
+  const int b = tile / p.Hv, h = tile - b * p.Hv, hk = h / (p.Hv / p.Hk);
+  if (p.mask != nullptr && p.mask[b] == 0) return;
+  const int r0 = 16 * warp + g, r1 = r0 + 8;
+  float2 S[2][G::NSPAN][8];
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+    for (int hh = 0; hh < G::NSPAN; ++hh)
+#pragma unroll
+      for (int e2 = 0; e2 < 8; ++e2) S[rr][hh][e2] = make_float2(0.0f, 0.0f);
+  if (p.S_in != nullptr && warp < G::NRB) {
+    const float *src = p.S_in + static_cast<size_t>(tile) * D * D;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+      for (int hh = 0; hh < G::NSPAN; ++hh) {
+        if (!chunk_valid<D>(t)) continue;
+        const float4 *row = reinterpret_cast<const float4 *>(
+            src + static_cast<size_t>(r0 + 8 * rr) * D + frag_col(hh, t, 0));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 v = row[u];
+          S[rr][hh][2 * u] = make_float2(v.x, v.y);
+          S[rr][hh][2 * u + 1] = make_float2(v.z, v.w);
+        }
+      }
+  }
+  const IT *q = static_cast<const IT *>(p.q), *k = static_cast<const IT *>(p.k);
+  const IT *v = static_cast<const IT *>(p.v);
+  const size_t tokB = static_cast<size_t>(p.B);
+  auto qk_at = [&](int tt) { return ((tt * tokB + b) * p.Hk + hk) * D; };
+  auto hv_at = [&](int tt) { return (tt * tokB + b) * p.Hv + h; };
+  // thread j < D carries channel j of the next token's inputs
+  float nq = 0.0f, nk = 0.0f, nv = 0.0f, na = 0.0f;
+  if (tid < D && p.T > 0) {
+    nq = to_f(q[qk_at(0) + tid]);
+    nk = to_f(k[qk_at(0) + tid]);
+    nv = to_f(v[hv_at(0) * D + tid]);
+    na = KDA ? p.alpha[hv_at(0) * D + tid] : 0.0f;
+  }
+  for (int tt = 0; tt < p.T; ++tt) {
+    if (tid < D) {
+      x.qf[tid] = nq;
+      x.kf[tid] = nk;
+      x.vf[tid] = nv;
+      if (KDA) x.G[tid] = na;
+      if (tt + 1 < p.T) {
+        nq = to_f(q[qk_at(tt + 1) + tid]);
+        nk = to_f(k[qk_at(tt + 1) + tid]);
+        nv = to_f(v[hv_at(tt + 1) * D + tid]);
+        if (KDA) na = p.alpha[hv_at(tt + 1) * D + tid];
+      }
+    }
+    __syncthreads();
+    if (warp < G::NRB) {
+      const float a0 = KDA ? 1.0f : p.alpha[hv_at(tt)];
+      const float beta = p.beta[hv_at(tt)];
+      float y0 = 0.0f, y1 = 0.0f;
+#pragma unroll
+      for (int hh = 0; hh < G::NSPAN; ++hh) {
+        if (!chunk_valid<D>(t)) continue;
+        const float4 *k4 = reinterpret_cast<const float4 *>(&x.kf[frag_col(hh, t, 0)]);
+        const float4 *a4 = reinterpret_cast<const float4 *>(&x.G[frag_col(hh, t, 0)]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 kk = k4[u];
+          const float4 aa = KDA ? a4[u] : make_float4(a0, a0, a0, a0);
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            float2 &sa = S[rr][hh][2 * u], &sb = S[rr][hh][2 * u + 1];
+            sa = __fmul2_rn(sa, make_float2(aa.x, aa.y));
+            sb = __fmul2_rn(sb, make_float2(aa.z, aa.w));
+            float &y = rr ? y1 : y0;
+            y = fmaf(sa.x, kk.x, y);
+            y = fmaf(sa.y, kk.y, y);
+            y = fmaf(sb.x, kk.z, y);
+            y = fmaf(sb.y, kk.w, y);
+          }
+        }
+      }
+      y0 += __shfl_xor_sync(kFull, y0, 1);
+      y1 += __shfl_xor_sync(kFull, y1, 1);
+      y0 += __shfl_xor_sync(kFull, y0, 2);
+      y1 += __shfl_xor_sync(kFull, y1, 2);
+      const float d0 = beta * (x.vf[r0] - y0), d1 = beta * (x.vf[r1] - y1);
+      float o0 = 0.0f, o1 = 0.0f;
+#pragma unroll
+      for (int hh = 0; hh < G::NSPAN; ++hh) {
+        if (!chunk_valid<D>(t)) continue;
+        const float4 *k4 = reinterpret_cast<const float4 *>(&x.kf[frag_col(hh, t, 0)]);
+        const float4 *q4 = reinterpret_cast<const float4 *>(&x.qf[frag_col(hh, t, 0)]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 kk = k4[u], qq = q4[u];
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const float dd = rr ? d1 : d0;
+            float2 &sa = S[rr][hh][2 * u], &sb = S[rr][hh][2 * u + 1];
+            sa = __ffma2_rn(make_float2(dd, dd), make_float2(kk.x, kk.y), sa);
+            sb = __ffma2_rn(make_float2(dd, dd), make_float2(kk.z, kk.w), sb);
+            float &o = rr ? o1 : o0;
+            o = fmaf(sa.x, qq.x, o);
+            o = fmaf(sa.y, qq.y, o);
+            o = fmaf(sb.x, qq.z, o);
+            o = fmaf(sb.y, qq.w, o);
+          }
+        }
+      }
+      o0 += __shfl_xor_sync(kFull, o0, 1);
+      o1 += __shfl_xor_sync(kFull, o1, 1);
+      o0 += __shfl_xor_sync(kFull, o0, 2);
+      o1 += __shfl_xor_sync(kFull, o1, 2);
+      if (p.out != nullptr && t == 0) {
+        st_out(p.out, static_cast<size_t>(hv_at(tt)) * D + r0, o0, p.out_bf16);
+        st_out(p.out, static_cast<size_t>(hv_at(tt)) * D + r1, o1, p.out_bf16);
+      }
+    }
+    __syncthreads();
+  }
+  quantize_tile<D>(s, reinterpret_cast<double *>(qscr),
+                   reinterpret_cast<float *>(qscr + G::NRB * D * 8), S,
+                   p.records + static_cast<size_t>(tile) * p.L.bytes, p.L, p.K, p.smooth);
+  if (tid == 0) p.buf_n[tile] = 0;
+}
+
 // ---------------------------------------------------------------------------
 // Launch plumbing
 // ---------------------------------------------------------------------------
@@ -1828,6 +1969,17 @@ cudaError_t init_t(const KParams &p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <int D, bool BF16, bool KDA>
+cudaError_t prefill_t(const KParams &p, cudaStream_t st) {
+  static LaunchInfo cache[32][kMaxComp + 1];
+  const size_t smem = D * D + sizeof(Scratch<D, false>);
+  LaunchInfo li;
+  cudaError_t e = prepare(prefill_kernel<D, BF16, KDA>, smem, smem, p.K, cache, li);
+  if (e != cudaSuccess) return e;
+  prefill_kernel<D, BF16, KDA><<<p.B * p.Hv, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
 template <template <int, bool, bool> class F>
 cudaError_t dispatch3(const KParams &p, cudaStream_t s) {
   const bool bf = p.in_bf16 != 0, kda = p.gate != 0;
@@ -1857,6 +2009,10 @@ template <int D, bool BF, bool KDA>
 struct DequantF {
   static cudaError_t run(const KParams &p, cudaStream_t s) { return fold_t<D, BF, KDA, 1>(p, s); }
 };
+template <int D, bool BF, bool KDA>
+struct PrefillF {
+  static cudaError_t run(const KParams &p, cudaStream_t s) { return prefill_t<D, BF, KDA>(p, s); }
+};
 
 }  // namespace
 
@@ -1865,6 +2021,7 @@ cudaError_t launch_flush(const KParams &p, cudaStream_t s) { return dispatch3<Fl
 cudaError_t launch_dequantize(const KParams &p, cudaStream_t s) {
   return dispatch3<DequantF>(p, s);
 }
+cudaError_t launch_prefill(const KParams &p, cudaStream_t s) { return dispatch3<PrefillF>(p, s); }
 cudaError_t launch_init(const KParams &p, cudaStream_t s) {
   if (p.d == 32) return init_t<32>(p, s);
   if (p.d == 64) return init_t<64>(p, s);

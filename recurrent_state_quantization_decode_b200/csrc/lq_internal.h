@@ -45,6 +45,7 @@ struct KParams {
   const float *S_in;    // init: fp32 states to quantize
   float *S_out;         // dequantize: fp32 states written
   int include_buffer;   // dequantize: advance the base state by the buffered tokens
+  int T;                // prefill: prompt tokens
   uint32_t wait_limit;  // decode: polls of a bounded mbarrier wait before it expires
   int withhold;         // decode, testing only: CTA 0 issues no copies for its first slot
 };
@@ -53,6 +54,7 @@ constexpr uint32_t kWaitLimitDefault = 1u << 24;
 
 cudaError_t launch_decode(const KParams &p, cudaStream_t stream);
 cudaError_t launch_init(const KParams &p, cudaStream_t stream);
+cudaError_t launch_prefill(const KParams &p, cudaStream_t stream);
 cudaError_t launch_flush(const KParams &p, cudaStream_t stream);
 cudaError_t launch_dequantize(const KParams &p, cudaStream_t stream);
 cudaError_t launch_fp32_step(const KParams &p, float *S, cudaStream_t stream);
