@@ -233,6 +233,23 @@ lq_status lq_test_decode_step_timeout(const lq_config *cfg, const void *q, const
                                       const lq_state *st, void *out, uint32_t wait_limit,
                                       void *stream);
 
+/* Prefix-cache checkpoints (news article on LeapQuant, paragraph 5: one
+ * state checkpoint per 1,024 tokens for prefix caching).  The checkpoint of
+ * sequence b is the Hv records of its tiles taken on a window boundary
+ * (buf_n == 0; call lq_window_flush first when off one), so restoring it
+ * gives a state that decodes on bit for bit.  pool: device memory of
+ * num_slots x Hv x layout.record_bytes, 16-byte aligned; slot s holds one
+ * sequence's checkpoint.  slots: device [B] int32, the pool slot of each
+ * sequence, -1 to skip it.  One checkpoint costs Hv x record_bytes (19,472 B
+ * per head at d = 128, K = 4) against Hv x 65,536 B for an fp32 state.
+ * save: a tile off a boundary, or a slot >= num_slots, is skipped and sets
+ * LQ_ERR_DEVICE_BOUNDS in the error word.  restore: the records are copied
+ * in and buf_n is set to 0 (a slot >= num_slots likewise). */
+lq_status lq_checkpoint_save(const lq_config *cfg, const lq_state *st, const int32_t *slots,
+                             void *pool, int32_t num_slots, void *stream);
+lq_status lq_checkpoint_restore(const lq_config *cfg, const void *pool, int32_t num_slots,
+                                const int32_t *slots, const lq_state *st, void *stream);
+
 /* Fold a partially filled window now (0 < buf_n < W) for the selected
  * sequences, exactly as the boundary fold does (news article, paragraph 3:
  * reconstruct and quantize at the boundary).  Used at the end of a sequence

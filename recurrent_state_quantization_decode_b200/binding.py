@@ -34,7 +34,8 @@ EXPORTED = ("lq_version", "lq_status_string", "lq_state_layout", "lq_state_bytes
             "lq_state_init", "lq_decode_step", "lq_decode_step_host",
             "lq_decode_step_host_noalloc", "lq_window_flush",
             "lq_fp32_decode_step", "lq_state_dequantize", "lq_get_last_error",
-            "lq_test_decode_step_timeout", "lq_prefill")
+            "lq_test_decode_step_timeout", "lq_prefill", "lq_checkpoint_save",
+            "lq_checkpoint_restore")
 
 
 class lq_config(ctypes.Structure):
@@ -79,6 +80,8 @@ _sig = {
                                     ctypes.c_int),
     "lq_prefill": ([_CFG, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _ST, _P, _P, _P],
                    ctypes.c_int),
+    "lq_checkpoint_save": ([_CFG, _ST, _P, _P, ctypes.c_int32, _P], ctypes.c_int),
+    "lq_checkpoint_restore": ([_CFG, _P, ctypes.c_int32, _P, _ST, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _sig.items():
     _f = getattr(_lib, _name)
@@ -183,6 +186,23 @@ def lq_prefill(cfg, q, k, v, alpha, beta, T: int, S0, state: lq_state, out=None,
     _check(_lib.lq_prefill(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
                            _ptr(beta), ctypes.c_int32(T), _ptr(S0), ctypes.byref(state),
                            _ptr(out), _ptr(mask), _stream(stream)), "lq_prefill")
+
+
+def lq_checkpoint_save(cfg, state: lq_state, slots, pool, num_slots: int,
+                       stream=None) -> None:
+    """Copy the records of the sequences with slots[b] >= 0 into pool slot
+    slots[b] (tiles must be on a window boundary)."""
+    _check(_lib.lq_checkpoint_save(ctypes.byref(cfg), ctypes.byref(state), _ptr(slots),
+                                   _ptr(pool), ctypes.c_int32(num_slots), _stream(stream)),
+           "lq_checkpoint_save")
+
+
+def lq_checkpoint_restore(cfg, pool, num_slots: int, slots, state: lq_state,
+                          stream=None) -> None:
+    """Copy pool slot slots[b] into sequence b's records (buf_n = 0)."""
+    _check(_lib.lq_checkpoint_restore(ctypes.byref(cfg), _ptr(pool), ctypes.c_int32(num_slots),
+                                      _ptr(slots), ctypes.byref(state), _stream(stream)),
+           "lq_checkpoint_restore")
 
 
 def lq_test_decode_step_timeout(cfg, q, k, v, alpha, beta, state: lq_state, out,

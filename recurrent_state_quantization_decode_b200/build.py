@@ -17,8 +17,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libleapquant.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("lq_decode.cu", "lq_fp32.cu", "lq_capi.cu", "lq_noalloc.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, "lq_internal.h"), os.path.join(INCLUDE, "leapquant.h")]
+SOURCES = [os.path.join(CSRC, f) for f in ("lq_decode.cu", "lq_fp32.cu", "lq_checkpoint.cu",
+                                            "lq_capi.cu", "lq_noalloc.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, h) for h in ("lq_internal.h", "lq_checkpoint.h")] + \
+    [os.path.join(INCLUDE, "leapquant.h")]
 
 
 def nvcc() -> str:

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/leapquant.h"
+#include "lq_checkpoint.h"
 #include "lq_internal.h"
 
 namespace {
@@ -207,6 +208,33 @@ lq_status lq_prefill(const lq_config *cfg, const void *q, const void *k, const v
   p.out = out;
   p.mask = mask;
   return from_cuda(lq::launch_prefill(p, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+lq_status checkpoint(bool save, const lq_config *cfg, const lq_state *st, const int32_t *slots,
+                     const void *pool, int32_t num_slots, void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if (slots == nullptr || pool == nullptr || num_slots < 0) return LQ_ERR_INVALID_ARG;
+  if (!aligned16(pool) || !aligned_to(slots, 4)) return LQ_ERR_MISALIGNED;
+  if (cfg->batch == 0) return LQ_OK;
+  const lq::RecLayout L = lq::record_layout(cfg->d, cfg->n_comp);
+  return from_cuda(lq::launch_checkpoint(
+      save, cfg->batch, cfg->num_v_heads, L.bytes, num_slots, slots,
+      static_cast<uint8_t *>(st->records), static_cast<uint8_t *>(const_cast<void *>(pool)),
+      st->buf_n, st->err, lq::kErrBadPhase, static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+lq_status lq_checkpoint_save(const lq_config *cfg, const lq_state *st, const int32_t *slots,
+                             void *pool, int32_t num_slots, void *stream) {
+  return checkpoint(true, cfg, st, slots, pool, num_slots, stream);
+}
+
+lq_status lq_checkpoint_restore(const lq_config *cfg, const void *pool, int32_t num_slots,
+                                const int32_t *slots, const lq_state *st, void *stream) {
+  return checkpoint(false, cfg, st, slots, pool, num_slots, stream);
 }
 
 lq_status lq_test_decode_step_timeout(const lq_config *cfg, const void *q, const void *k,

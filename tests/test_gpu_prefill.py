@@ -90,3 +90,47 @@ def test_prefill_of_zero_tokens_is_init():
     torch.cuda.synchronize()
     assert torch.equal(a.records, b.records)
     assert B.lq_get_last_error(b.st) == B.LQ_OK
+
+
+def test_checkpoint_pool_roundtrip_errors_and_accounting():
+    """lq_checkpoint_save / restore: a round trip is bit-exact and decodes on
+    identically; a tile off a window boundary or a slot past the pool is
+    refused through the error word; one checkpoint costs Hv records."""
+    w = wl.Workload("ck", 4, 2, 4, 128, wl.GATE_SCALAR, True, 1)
+    rng = np.random.default_rng(33)
+    S0, _, _ = wl.initial_states(rng, w.tiles, w.d, w.d)
+    ti = wl.token_inputs(rng, w, 3)
+    cfg = B.config_for(w)
+    L = B.lq_state_layout(cfg)
+    pool = torch.zeros(2 * w.num_v_heads * L.record_bytes, dtype=torch.uint8, device="cuda")
+    # one checkpoint: Hv records against Hv fp32 states
+    assert L.record_bytes == 19472
+    assert round(65536 / L.record_bytes, 2) == 3.37
+    ds = B.DeviceState(cfg)
+    B.lq_state_init(cfg, torch.from_numpy(S0).cuda(), ds.st)
+    slots = torch.tensor([1, -1, 0, -1], dtype=torch.int32, device="cuda")
+    B.lq_checkpoint_save(cfg, ds.st, slots, pool, 2)
+    assert B.lq_get_last_error(ds.st) == B.LQ_OK
+    rec = ds.record_view()
+    pv = pool.view(2, w.num_v_heads, L.record_bytes)
+    hv = w.num_v_heads
+    assert torch.equal(pv[1], rec[0:hv]) and torch.equal(pv[0], rec[2 * hv:3 * hv])
+    # restore into a fresh state: both decode the next tokens identically
+    ds2 = B.DeviceState(cfg)
+    B.lq_state_init(cfg, torch.zeros_like(torch.from_numpy(S0)).cuda(), ds2.st)
+    B.lq_checkpoint_restore(cfg, pool, 2, slots, ds2.st)
+    dev = P.DeviceInputs(ti, True)
+    act = torch.tensor([1, 0, 1, 0], dtype=torch.int32, device="cuda")
+    o1 = torch.empty((w.batch, hv, w.d), device="cuda")
+    o2 = torch.empty_like(o1)
+    for t in range(2):
+        B.lq_decode_step(cfg, *dev.token(t), ds.st, o1, active=act)
+        B.lq_decode_step(cfg, *dev.token(t), ds2.st, o2, active=act)
+        assert torch.equal(o1[0], o2[0]) and torch.equal(o1[2], o2[2])
+    # sequence 0 is now off a window boundary: its save is refused
+    B.lq_checkpoint_save(cfg, ds.st, slots, pool, 2)
+    assert B.lq_get_last_error(ds.st) == B.LQ_ERR_DEVICE_BOUNDS
+    # a slot past the pool is refused too
+    bad = torch.tensor([5, -1, -1, -1], dtype=torch.int32, device="cuda")
+    B.lq_checkpoint_restore(cfg, pool, 2, bad, ds2.st)
+    assert B.lq_get_last_error(ds2.st) == B.LQ_ERR_DEVICE_BOUNDS

@@ -4,10 +4,10 @@ tokens) at a reduced size, through the C-ABI decode step.
 
 It checks three things:
 
-- Checkpoint / resume: a record copied at a 1,024-token boundary (news
+- Checkpoint / resume: lq_checkpoint_save at a 1,024-token boundary (news
   article, paragraph 5: one state checkpoint per 1,024 tokens for prefix
-  caching) restores into a fresh state, and replaying the same tokens
-  reproduces the original outputs bit for bit.
+  caching), lq_checkpoint_restore into a fresh state, and replaying the same
+  tokens reproduces the original outputs bit for bit.
 - Drift against the exact recurrence: on sampled tiles (the longest
   sequences among them) the int8-state outputs are compared with the exact
   fp64 recurrence over the whole decode.  The drift of LeapQuant (W = 16,
@@ -44,6 +44,10 @@ def _binding():
     from recurrent_state_quantization_decode_b200 import binding
 
     return binding
+
+
+def ds_layout_record(B, cfg) -> int:
+    return B.lq_state_layout(cfg).record_bytes
 
 
 def _normwise(a, b):
@@ -86,7 +90,10 @@ def test_long_ragged_decode_checkpoint_resume_and_drift():
     smp_hk = smp_h // (HV // HK)
     host_inputs = {n: [] for n in ("q", "k", "v", "alpha", "beta")}
     out = torch.empty((B_SEQ, HV, D), device="cuda")
-    checkpoint = None
+    # a one-slot checkpoint pool; sequence rb's checkpoint goes to slot 0
+    pool = torch.zeros(HV * ds_layout_record(B, cfg), dtype=torch.uint8, device="cuda")
+    slots = torch.full((B_SEQ,), -1, dtype=torch.int32, device="cuda")
+    slots[rb] = 0
     dev_chunks = []
     for c0 in range(0, T, CHUNK):
         ti = wl.token_inputs(rng, w, min(CHUNK, T - c0))
@@ -120,15 +127,14 @@ def test_long_ragged_decode_checkpoint_resume_and_drift():
             if t == ck_step:
                 ds = states["leapquant"]
                 assert int(ds.buf_n[rb * HV]) == 0          # on a window boundary
-                checkpoint = ds.record_view()[rb_tiles].clone()
+                B.lq_checkpoint_save(cfg, ds.st, slots, pool, 1)
     for ds in states.values():
         assert B.lq_get_last_error(ds.st) == B.LQ_OK
 
     # resume from the checkpoint in a fresh state: only sequence rb is active
     ds2 = B.DeviceState(cfg)
     B.lq_state_init(cfg, S0_dev, ds2.st)
-    ds2.record_view()[rb_tiles] = checkpoint
-    ds2.buf_n.zero_()
+    B.lq_checkpoint_restore(cfg, pool, 1, slots, ds2.st)
     only = torch.zeros(B_SEQ, dtype=torch.int32, device="cuda")
     only[rb] = 1
     replay = torch.full_like(rb_hist, float("nan"))
