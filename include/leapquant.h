@@ -1,7 +1,10 @@
 /*
  * leapquant.h - C ABI of libleapquant.so: the per-token decode step of a
  * Gated DeltaNet (GDN) / Kimi Delta Attention (KDA) layer whose recurrent
- * state is stored in int8, following LeapQuant.
+ * state is stored in int8, following LeapQuant, with the calls around it:
+ * state init, a prefill that ends in the quantizer, partial-window flush,
+ * prefix-cache checkpoints, dequantization and the fp32-state comparison
+ * step.
  *
  * Method sources (page title, section):
  *  - "LeapQuant: Training-Free 8-bit Quantization for Linear Attention
@@ -38,15 +41,18 @@
  *           fp32 gates alpha_i.
  *  buf_n    [B][Hv] int32 tokens buffered in the current window (0..W-1
  *           between calls).
- *  err      one int32 device error word (bit 0: a corrupt buf_n was seen;
- *           bit 1: a bounded wait on a copy expired).
+ *  err      one int32 device error word (bit 0: a corrupt buf_n was seen,
+ *           or a checkpoint copy was refused; bit 1: a bounded wait on a
+ *           copy expired).
  * The layout is public: a checkpoint of a tile at a window boundary is a copy
  * of its record.
  *
  * Conventions for every call:
  *  - All pointers in lq_state and all tensor arguments are device pointers
  *    unless the name says host; the library allocates nothing and keeps no
- *    global state.  `stream` is a cudaStream_t (NULL = legacy default).
+ *    global state, except the fixed staging array of
+ *    lq_decode_step_host_noalloc.  `stream` is a cudaStream_t (NULL = legacy
+ *    default).
  *  - Argument errors are detected on the host before anything is launched,
  *    and reported synchronously: LQ_ERR_INVALID_ARG (null pointer, bad
  *    shape), LQ_ERR_UNSUPPORTED (d not in {32, 64, 128}, W not in 1..16,
