@@ -450,6 +450,26 @@ __device__ __forceinline__ void load_codes(const uint8_t *codes, uint4 (&A)[2][F
 // Element e (0..15) of span h of row rr in a float2 register tile.
 #define SX(rr, h, e) ((((e) & 1) != 0) ? S[rr][h][(e) >> 1].y : S[rr][h][(e) >> 1].x)
 
+// f(entry of row r0, entry of row r1) at column slot e (0..15) of span h of
+// this lane's fragment, for a runtime (h, e) that every calling lane shares:
+// a switch reaches the one register pair instead of testing all 32 slots.
+#define LQ_SLOT(H, E) \
+  case (H) * 16 + (E): f(SX(0, H, E), SX(1, H, E)); break;
+#define LQ_SPAN(H) \
+  LQ_SLOT(H, 0) LQ_SLOT(H, 1) LQ_SLOT(H, 2) LQ_SLOT(H, 3) LQ_SLOT(H, 4) LQ_SLOT(H, 5) \
+  LQ_SLOT(H, 6) LQ_SLOT(H, 7) LQ_SLOT(H, 8) LQ_SLOT(H, 9) LQ_SLOT(H, 10) LQ_SLOT(H, 11) \
+  LQ_SLOT(H, 12) LQ_SLOT(H, 13) LQ_SLOT(H, 14) LQ_SLOT(H, 15)
+template <int NSPAN, class F>
+__device__ __forceinline__ void at_slot(float2 (&S)[2][NSPAN][8], int h, int e, F &&f) {
+  if constexpr (NSPAN > 1) {
+    switch (h * 16 + e) { LQ_SPAN(0) LQ_SPAN(1) default: break; }
+  } else {
+    switch (h * 16 + e) { LQ_SPAN(0) default: break; }
+  }
+}
+#undef LQ_SPAN
+#undef LQ_SLOT
+
 // The fp32 state of the thread's block (warps that own rows), as float2 pairs
 // along the columns:
 //   S_ij = sigma_i code_ij (m_j Gamma_j) + sum_{s < nent} d_s[i] kt_s[j]
@@ -558,14 +578,10 @@ __device__ __forceinline__ void build_state(const SC &x, const float *kt,
       if (((jc & 63) >> 4) == t && chunk_valid<D>(t)) {
         const float gj = x.G[jc];
         const float a0 = rcv[c * D + r0] * gj, a1 = rcv[c * D + r1] * gj;
-#pragma unroll
-        for (int h = 0; h < G::NSPAN; ++h)
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (frag_col(h, t, e) == jc) {
-              SX(0, h, e) += a0;
-              SX(1, h, e) += a1;
-            }
+        at_slot<G::NSPAN>(S, jc >> 6, jc & 15, [&](float &u0, float &u1) {
+          u0 += a0;
+          u1 += a1;
+        });
       }
     }
   }
@@ -702,16 +718,12 @@ __device__ void quantize_tile(SC &s, double *colpart, float *colmax,
         } else {
           const int jc = id - D;
           if (((jc & 63) >> 4) == t && chunk_valid<D>(t)) {
-#pragma unroll
-            for (int h = 0; h < G::NSPAN; ++h)
-#pragma unroll
-              for (int e = 0; e < 16; ++e)
-                if (frag_col(h, t, e) == jc) {
-                  s.line[r0] = SX(0, h, e);
-                  s.line[r1] = SX(1, h, e);
-                  SX(0, h, e) = 0.0f;
-                  SX(1, h, e) = 0.0f;
-                }
+            at_slot<G::NSPAN>(S, jc >> 6, jc & 15, [&](float &u0, float &u1) {
+              s.line[r0] = u0;
+              s.line[r1] = u1;
+              u0 = 0.0f;
+              u1 = 0.0f;
+            });
           }
         }
       }
