@@ -37,8 +37,13 @@
 //    tile while others finish the current one, and every thread waits on the
 //    slot's mbarrier itself.
 //  * On the boundary token the fp32 state S = S0 diag(Gamma) + sum d_s kt_s^T
-//    is built in registers, in the same fragment layout as the codes, and the
-//    quantizer (compensator lines, smoothing, per-row int8) runs on it.
+//    is built in registers, in the same fragment layout as the codes: the
+//    dequantized base, then (d >= 64) the rank-W update on the tf32 tensor
+//    path with each operand split into hi and lo parts, whose accumulator
+//    fragment is that layout.  The quantizer (compensator lines, smoothing,
+//    per-row int8) then runs on it.
+//  * prefill_kernel runs the exact recurrence over a prompt with the state in
+//    the same registers and ends in the same quantizer.
 //
 // Fragment layout: warp w < D/16 owns state rows 16w..16w+15; lane (g = lane/4,
 // t = lane%4) owns rows 16w+g and 16w+g+8 and, in every 64-column span h, the
@@ -1085,13 +1090,20 @@ __device__ __forceinline__ void channel_chunk_fast(const KParams &p, TK &x,
 }
 
 // One token for one staged tile: outputs, buffer append, and on the W-th token
-// the fold and requantization.  Three phases separated by CTA barriers:
+// the fold and requantization.
+// GDN with bf16 inputs (one CTA barrier; returns false if the CTA aborts):
+//  A  warp c < 2 NSPAN: k-chunk c's channels (gate product, x, chunk max,
+//     digits and scale); warp 2 NSPAN: the buffer coefficients c_s, a_s (bf16
+//     MMA); the other warps: their code fragments, then the row-compensator
+//     dots.  Then the barrier, after which the caller's refill runs.
+// General path (KDA, fp32 inputs), phases separated by CTA barriers:
 //  A  channel threads (one per key channel j): inputs, decay ratios applied to
 //     the buffered keys, Gamma, x = m o Gamma o {q, k} and its per-warp max;
 //     appends k_t and the KDA gate.  The other warps fetch their code
 //     fragments.
 //  B  channel threads: the int8 digits of x_q, x_k and the row-compensator
 //     dots; the other warps: the buffer coefficients c_s, a_s.
+// Both then run
 //  C  every row warp: y_q, y_k for its 16 rows on the int8 tensor path, then
 //     finishes its rows (buffer sums split over the 4 lanes of a row):
 //     d_t = beta (v - y_k - sum c_s d_s), o_t = y_q + sum a_s d_s + a_t d_t.
