@@ -256,6 +256,19 @@ lq_status lq_checkpoint_save(const lq_config *cfg, const lq_state *st, const int
 lq_status lq_checkpoint_restore(const lq_config *cfg, const void *pool, int32_t num_slots,
                                 const int32_t *slots, const lq_state *st, void *stream);
 
+/* Speculative decoding: drop the last drop[b] decoded tokens of sequence b
+ * (drop: device [B] int32, 0 = keep all).  Inside a window the record is
+ * fixed and the buffered tokens are appended entries (zhichai.net summary,
+ * "Abstract (translated)", item 1: outputs from the fixed low-bit state plus
+ * the buffer), so rejecting draft tokens only moves the window phase back
+ * and the state afterwards is exactly the one that never saw them.  This
+ * holds while no window boundary was crossed since the draft began: a drop
+ * larger than the tile's buffered count (or negative) is refused for that
+ * tile with LQ_ERR_DEVICE_BOUNDS in the error word.  The pages have no
+ * counterpart to this call. */
+lq_status lq_window_rewind(const lq_config *cfg, const lq_state *st, const int32_t *drop,
+                           void *stream);
+
 /* Fold a partially filled window now (0 < buf_n < W) for the selected
  * sequences, exactly as the boundary fold does (news article, paragraph 3:
  * reconstruct and quantize at the boundary).  Used at the end of a sequence

@@ -35,7 +35,7 @@ EXPORTED = ("lq_version", "lq_status_string", "lq_state_layout", "lq_state_bytes
             "lq_decode_step_host_noalloc", "lq_window_flush",
             "lq_fp32_decode_step", "lq_state_dequantize", "lq_get_last_error",
             "lq_test_decode_step_timeout", "lq_prefill", "lq_checkpoint_save",
-            "lq_checkpoint_restore")
+            "lq_checkpoint_restore", "lq_window_rewind")
 
 
 class lq_config(ctypes.Structure):
@@ -82,6 +82,7 @@ _sig = {
                    ctypes.c_int),
     "lq_checkpoint_save": ([_CFG, _ST, _P, _P, ctypes.c_int32, _P], ctypes.c_int),
     "lq_checkpoint_restore": ([_CFG, _P, ctypes.c_int32, _P, _ST, _P], ctypes.c_int),
+    "lq_window_rewind": ([_CFG, _ST, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _sig.items():
     _f = getattr(_lib, _name)
@@ -203,6 +204,12 @@ def lq_checkpoint_restore(cfg, pool, num_slots: int, slots, state: lq_state,
     _check(_lib.lq_checkpoint_restore(ctypes.byref(cfg), _ptr(pool), ctypes.c_int32(num_slots),
                                       _ptr(slots), ctypes.byref(state), _stream(stream)),
            "lq_checkpoint_restore")
+
+
+def lq_window_rewind(cfg, state: lq_state, drop, stream=None) -> None:
+    """Drop the last drop[b] decoded tokens of sequence b (inside a window)."""
+    _check(_lib.lq_window_rewind(ctypes.byref(cfg), ctypes.byref(state), _ptr(drop),
+                                 _stream(stream)), "lq_window_rewind")
 
 
 def lq_test_decode_step_timeout(cfg, q, k, v, alpha, beta, state: lq_state, out,

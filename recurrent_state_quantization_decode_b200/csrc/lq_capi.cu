@@ -237,6 +237,17 @@ lq_status lq_checkpoint_restore(const lq_config *cfg, const void *pool, int32_t 
   return checkpoint(false, cfg, st, slots, pool, num_slots, stream);
 }
 
+lq_status lq_window_rewind(const lq_config *cfg, const lq_state *st, const int32_t *drop,
+                           void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if (drop == nullptr) return LQ_ERR_INVALID_ARG;
+  if (!aligned_to(drop, 4)) return LQ_ERR_MISALIGNED;
+  return from_cuda(lq::launch_rewind(cfg->batch, cfg->num_v_heads, drop, st->buf_n, st->err,
+                                     lq::kErrBadPhase, static_cast<cudaStream_t>(stream)));
+}
+
 lq_status lq_test_decode_step_timeout(const lq_config *cfg, const void *q, const void *k,
                                       const void *v, const float *alpha, const float *beta,
                                       const lq_state *st, void *out, uint32_t wait_limit,

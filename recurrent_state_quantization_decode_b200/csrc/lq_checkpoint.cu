@@ -1,4 +1,5 @@
-// Prefix-cache checkpoints of the int8 state: a checkpoint of a sequence is a
+// Prefix-cache checkpoints of the int8 state, and rollback inside a window.
+// A checkpoint of a sequence is a
 // copy of its tile records taken at a window boundary, when the in-window
 // buffer is empty (news article on LeapQuant, paragraph 5: one state
 // checkpoint per 1,024 tokens for prefix caching, at 1.19 bytes per value).
@@ -40,7 +41,32 @@ __global__ void __launch_bounds__(kCopyThreads)
   }
 }
 
+// One thread per tile.  Within a window the record is fixed and the
+// buffered tokens are appended entries, so dropping the last ones is exact.
+__global__ void rewind_kernel(int tiles, int Hv, const int32_t *drop, int32_t *buf_n,
+                              int32_t *err, int err_bad_phase) {
+  const int tile = blockIdx.x * blockDim.x + threadIdx.x;
+  if (tile >= tiles) return;
+  const int k = drop[tile / Hv];
+  if (k == 0) return;
+  const int n = buf_n[tile];
+  if (k < 0 || k > n) {
+    atomicOr(err, err_bad_phase);
+    return;
+  }
+  buf_n[tile] = n - k;
+}
+
 }  // namespace
+
+cudaError_t launch_rewind(int B, int Hv, const int32_t *drop, int32_t *buf_n, int32_t *err,
+                          int err_bad_phase, cudaStream_t stream) {
+  const int tiles = B * Hv;
+  if (tiles == 0) return cudaSuccess;
+  rewind_kernel<<<(tiles + 255) / 256, 256, 0, stream>>>(tiles, Hv, drop, buf_n, err,
+                                                         err_bad_phase);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_checkpoint(bool save, int B, int Hv, int record_bytes, int num_slots,
                               const int32_t *slots, uint8_t *records, uint8_t *pool,

@@ -19,4 +19,11 @@ cudaError_t launch_checkpoint(bool save, int B, int Hv, int record_bytes, int nu
                               int32_t *buf_n, int32_t *err, int err_bad_phase,
                               cudaStream_t stream);
 
+// Speculative-decoding rollback: drop the last drop[b] buffered tokens of
+// every tile of sequence b (buf_n -= drop[b]); drop[b] > buf_n (a fold
+// happened since the draft began) or drop[b] < 0 sets `err_bad_phase` and
+// leaves the tile unchanged.
+cudaError_t launch_rewind(int B, int Hv, const int32_t *drop, int32_t *buf_n, int32_t *err,
+                          int err_bad_phase, cudaStream_t stream);
+
 }  // namespace lq
