@@ -198,7 +198,7 @@ struct Scratch : KtArea<D, KT> {
   alignas(16) float invm[FG<D>::PADW];             // 1 / m (new smoothing factors)
   alignas(16) float line[D];                       // the compensator line being extracted
   alignas(16) double rowE[D];
-  double pbest[kWarps];              // per-warp partial argmax of the line energies
+  unsigned long long pkey[kWarps];   // per-warp best selection key of the line energies
   int pid[kWarps];
   int abort;
   int done[3];  // warps finished with each ring slot (GDN-bf16 path)
@@ -592,12 +592,22 @@ __device__ __forceinline__ void build_state(const SC &x, const float *kt,
   }
 }
 
+// Selection key of a candidate line for the greedy picks: 0 for a taken line,
+// else 1 + the bit pattern of its fp64 energy, which orders like the value for
+// a non-negative double; an energy that the subtractions of removed lines
+// left below zero counts as zero.
+__device__ __forceinline__ unsigned long long line_key(double e, bool taken) {
+  if (taken) return 0ull;
+  return (e > 0.0 ? static_cast<unsigned long long>(__double_as_longlong(e)) : 0ull) + 1ull;
+}
+
 // Quantize the state held in registers (fragment layout) into the record at
 // rec (global):
 //  1. K times: the untaken line (row or column) of the largest fp64 energy of
 //     the residual (ties: lower id; rows are ids 0..D-1, columns D..2D-1) is
 //     stored as an fp32 compensator vector and zeroed; the energies of the
-//     crossing lines lose the removed squares;
+//     crossing lines lose the removed squares (an energy that these
+//     subtractions leave below zero counts as zero);
 //  2. m_j from the residual's column max a_j: 1 if smoothing is off or
 //     a_j < FLT_MIN, else sqrt(a_j) or a_j;
 //  3. per row: x = (R_ij * (1/m_j)) * (127/b_i) with b_i the row max of
@@ -659,64 +669,60 @@ __device__ void quantize_tile(SC &s, double *colpart, float *colmax,
       for (int w = 0; w < G::NRB; ++w) eCol += colpart[w * D + tid];
     }
     for (int c = 0; c < K; ++c) {
-      // partial argmax over this thread's two candidates, then over the warp
+      // argmax over this thread's two candidates (the row wins a tie: lower
+      // id), then over the warp: the largest key, then the lowest id holding it
       if (warp < (D + 31) / 32) {
-        double best = -1.0;
-        int bid = 0x7fffffff;
-        if (tid < D) {
-          if (!tRow) {
-            best = eRow;
-            bid = tid;
-          }
-          if (!tCol && eCol > best) {
-            best = eCol;
-            bid = D + tid;
-          }
+        const unsigned long long kr = line_key(eRow, tRow), kc = line_key(eCol, tCol);
+        unsigned long long key = kr;
+        int bid = tid;
+        if (kc > kr) {
+          key = kc;
+          bid = D + tid;
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const double ob = __shfl_xor_sync(kFull, best, o);
-          const int oid = __shfl_xor_sync(kFull, bid, o);
-          if (ob > best || (ob == best && oid < bid)) {
-            best = ob;
-            bid = oid;
-          }
-        }
+        const uint32_t khi = static_cast<uint32_t>(key >> 32), klo = static_cast<uint32_t>(key);
+        const uint32_t whi = __reduce_max_sync(kFull, khi);
+        const uint32_t wlo = __reduce_max_sync(kFull, khi == whi ? klo : 0u);
+        const uint32_t wid =
+            __reduce_min_sync(kFull, (khi == whi && klo == wlo) ? static_cast<uint32_t>(bid)
+                                                                : 0xffffffffu);
         if (lane == 0) {
-          s.pbest[warp] = best;
-          s.pid[warp] = bid;
+          s.pkey[warp] = (static_cast<unsigned long long>(whi) << 32) | wlo;
+          s.pid[warp] = static_cast<int>(wid);
         }
       }
       __syncthreads();
       // every thread combines the per-warp winners (same result everywhere)
       int id = 0x7fffffff;
       {
-        double best = -1.0;
+        unsigned long long best = 0ull;
 #pragma unroll
         for (int w = 0; w < (D + 31) / 32; ++w) {
-          const double e = s.pbest[w];
+          const unsigned long long k = s.pkey[w];
           const int i2 = s.pid[w];
-          if (e > best || (e == best && i2 < id)) {
-            best = e;
+          if (k > best || (k == best && i2 < id)) {
+            best = k;
             id = i2;
           }
         }
       }
-      // the owners of the line park its values in s.line and zero them
+      // the owners of the line park its values in s.line and zero them: a
+      // row lives in one warp (rows 16 w .. 16 w + 15), a column in all
       if (rows_here) {
         if (id < D) {
+          if (warp == (id >> 4)) {
 #pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            if ((rr ? r1 : r0) != id || !chunk_valid<D>(t)) continue;
+            for (int rr = 0; rr < 2; ++rr) {
+              if ((rr ? r1 : r0) != id || !chunk_valid<D>(t)) continue;
 #pragma unroll
-            for (int h = 0; h < G::NSPAN; ++h) {
-              float4 *dst = reinterpret_cast<float4 *>(&s.line[frag_col(h, t, 0)]);
+              for (int h = 0; h < G::NSPAN; ++h) {
+                float4 *dst = reinterpret_cast<float4 *>(&s.line[frag_col(h, t, 0)]);
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                dst[u] = make_float4(S[rr][h][2 * u].x, S[rr][h][2 * u].y, S[rr][h][2 * u + 1].x,
-                                     S[rr][h][2 * u + 1].y);
-                S[rr][h][2 * u] = make_float2(0.0f, 0.0f);
-                S[rr][h][2 * u + 1] = make_float2(0.0f, 0.0f);
+                for (int u = 0; u < 4; ++u) {
+                  dst[u] = make_float4(S[rr][h][2 * u].x, S[rr][h][2 * u].y, S[rr][h][2 * u + 1].x,
+                                       S[rr][h][2 * u + 1].y);
+                  S[rr][h][2 * u] = make_float2(0.0f, 0.0f);
+                  S[rr][h][2 * u + 1] = make_float2(0.0f, 0.0f);
+                }
               }
             }
           }
@@ -1397,8 +1403,11 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
     return true;
   }
 
-  // Window boundary: fold the W buffered tokens and requantize.
-  __syncthreads();
+  // Window boundary: fold the W buffered tokens and requantize.  A warp reads
+  // back only its own rows' d_t, written above by lanes of the same warp; the
+  // barriers below keep the codes and keys from being overwritten while
+  // another warp still needs them.
+  __syncwarp();
   float2 S[2][G::NSPAN][8];
   uint4 Af[2][G::NSPAN];
   if (warp < G::NRB) load_codes<D>(codes, Af);
