@@ -567,7 +567,8 @@ __device__ __forceinline__ void build_state(const SC &x, const float *kt,
   for (int c = 0; c < K; ++c) {
     const int id = rcid[c];
     if (id < D) {
-      if ((id == r0 || id == r1) && chunk_valid<D>(t)) {
+      // a row line lands in one warp (rows 16 w .. 16 w + 15)
+      if (warp == (id >> 4) && (id == r0 || id == r1) && chunk_valid<D>(t)) {
         const bool second = id == r1;
 #pragma unroll
         for (int h = 0; h < G::NSPAN; ++h)
