@@ -550,7 +550,8 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
         ms_e2e = max_over_ranks(start.elapsed_time(end), world, device)
         e2e = {"value": whole_job_rate(units_per_step, world, e2e_steps, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "path": ("lq_decode_step_host (pinned host q,k,v,alpha,beta in; o out), "
+               "path": ("lq_decode_step_host: pinned host q, k, v, alpha, beta read over "
+                        "the host link by the gather kernel, o back by cudaMemcpyAsync; "
                         f"{len(streams)} streams by layer index")}
 
     # prefill of one layer's tiles over a prompt, ending in the quantizer

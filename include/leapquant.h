@@ -185,12 +185,21 @@ lq_status lq_decode_step(const lq_config *cfg, const void *q, const void *k, con
                          const float *alpha, const float *beta, const lq_state *st, void *out,
                          const int32_t *active, void *stream);
 
-/* lq_decode_step with the token's inputs and output in HOST memory: copies
+/* lq_decode_step with the token's inputs and output in HOST memory: moves
  * q, k, v, alpha, beta to `staging` (device, layout.host_staging_bytes,
  * 16-byte aligned), runs the step, and copies o back to out_host, all
  * asynchronously on `stream` (the caller synchronizes before reading
- * out_host; pinned host memory makes the copies truly asynchronous).  The
- * state stays on the device.  active is a device pointer, as above. */
+ * out_host).  The state stays on the device.  active is a device pointer, as
+ * above.
+ *  - Inputs in pinned memory that the device maps at the same address
+ *    (cudaHostAlloc / cudaMallocHost memory under unified addressing, as the
+ *    driver reports through cudaPointerGetAttributes for both ends of the
+ *    input) are read by one gather kernel over the host link: a token's small
+ *    inputs then move without a copy-engine start-up per input.
+ *  - Any other host memory is copied with cudaMemcpyAsync (pageable memory
+ *    makes those copies synchronous with the host).
+ *  - The host buffers must hold the sizes listed for lq_decode_step and stay
+ *    unchanged until the stream reaches the step. */
 lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const void *k_host,
                               const void *v_host, const float *alpha_host,
                               const float *beta_host, const lq_state *st, void *out_host,

@@ -18,8 +18,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libleapquant.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("lq_decode.cu", "lq_fp32.cu", "lq_checkpoint.cu",
-                                            "lq_capi.cu", "lq_noalloc.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, h) for h in ("lq_internal.h", "lq_checkpoint.h")] + \
+                                            "lq_hostio.cu", "lq_capi.cu", "lq_noalloc.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, h) for h in ("lq_internal.h", "lq_checkpoint.h",
+                                                          "lq_hostio.h")] + \
     [os.path.join(INCLUDE, "leapquant.h")]
 
 

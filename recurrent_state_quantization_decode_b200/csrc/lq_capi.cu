@@ -9,6 +9,7 @@
 
 #include "../../include/leapquant.h"
 #include "lq_checkpoint.h"
+#include "lq_hostio.h"
 #include "lq_internal.h"
 
 namespace {
@@ -293,12 +294,21 @@ lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const vo
   uint8_t *da = dv + round256(nv);
   uint8_t *db = da + round256(na);
   uint8_t *dout = db + round256(nb);
-  if (cudaMemcpyAsync(dq, q_host, nq, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(dk, k_host, nq, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(dv, v_host, nv, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(da, alpha_host, na, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(db, beta_host, nb, cudaMemcpyHostToDevice, cs) != cudaSuccess)
-    return LQ_ERR_CUDA;
+  // Inputs in device-mapped pinned memory are read by one gather kernel over
+  // the host link; any other host memory goes through the copy engine.
+  const void *src[5] = {q_host, k_host, v_host, alpha_host, beta_host};
+  void *dst[5] = {dq, dk, dv, da, db};
+  const size_t bytes[5] = {nq, nq, nv, na, nb};
+  lq::GatherList gather{};
+  for (int i = 0; i < 5; ++i) {
+    if (const void *view = lq::device_view_of_host(src[i], bytes[i])) {
+      gather.seg[gather.n++] = lq::GatherSeg{view, dst[i], bytes[i]};
+    } else if (cudaMemcpyAsync(dst[i], src[i], bytes[i], cudaMemcpyHostToDevice, cs) !=
+               cudaSuccess) {
+      return LQ_ERR_CUDA;
+    }
+  }
+  if (lq::launch_gather(gather, cs) != cudaSuccess) return LQ_ERR_CUDA;
   KParams p = make_params(cfg, st);
   p.q = dq;
   p.k = dk;

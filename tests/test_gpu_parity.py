@@ -435,8 +435,23 @@ def test_bounded_wait_expiry_reports_timeout(bf16, gate):
     assert torch.isfinite(out).all()
 
 
-def test_host_entry_point_matches_device_entry_point():
-    w = wl.Workload("h", 4, 2, 4, 128, wl.GATE_SCALAR, True, 20)
+HOST_MODES = {
+    # inputs in pinned memory: the gather kernel reads them over the host link
+    "pinned": (wl.Workload("h", 4, 2, 4, 128, wl.GATE_SCALAR, True, 20), set("qkv") | {"alpha", "beta"}),
+    # pageable memory: every input goes through cudaMemcpyAsync
+    "pageable": (wl.Workload("h", 4, 2, 4, 128, wl.GATE_SCALAR, True, 20), set()),
+    # some of each in one call
+    "mixed": (wl.Workload("h", 4, 2, 4, 128, wl.GATE_SCALAR, True, 20), {"q", "v"}),
+    # 9 tiles: alpha and beta of 36 bytes (a ragged tail), placed 4 bytes off
+    # a 16-byte boundary in pinned memory (the bytewise path)
+    "ragged_misaligned": (wl.Workload("h9", 3, 1, 3, 64, wl.GATE_SCALAR, True, 20),
+                          set("qkv") | {"alpha", "beta"}),
+}
+
+
+@pytest.mark.parametrize("mode", sorted(HOST_MODES))
+def test_host_entry_point_matches_device_entry_point(mode):
+    w, pinned = HOST_MODES[mode]
     rng = np.random.default_rng(6)
     S0, _, _ = wl.initial_states(rng, w.tiles, w.d, w.d)
     ti = wl.token_inputs(rng, w, 20)
@@ -447,7 +462,20 @@ def test_host_entry_point_matches_device_entry_point():
     B.lq_state_init(cfg, S0_dev, a.st)
     B.lq_state_init(cfg, S0_dev, b.st)
     dev = P.DeviceInputs(ti, True)
-    host = {n: getattr(dev, n).cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
+    host = {}
+    for n in ("q", "k", "v", "alpha", "beta"):
+        x = getattr(dev, n).cpu()
+        if n in pinned and mode == "ragged_misaligned" and n in ("alpha", "beta"):
+            buf = torch.empty(x.numel() + 1, dtype=x.dtype).pin_memory()
+            view = buf[1:].view(x.shape)
+            view.copy_(x)
+            assert view.data_ptr() % 16 == 4
+            x = view
+        elif n in pinned:
+            x = x.pin_memory()
+        else:
+            assert not x.is_pinned()
+        host[n] = x
     staging = torch.empty(B.lq_state_layout(cfg).host_staging_bytes, dtype=torch.uint8,
                           device="cuda")
     out_d = torch.empty((w.batch, w.num_v_heads, w.d), device="cuda")
@@ -459,3 +487,4 @@ def test_host_entry_point_matches_device_entry_point():
         _sync()
         np.testing.assert_array_equal(out_h.numpy(), out_d.cpu().numpy())
     assert torch.equal(a.records, b.records)
+    assert B.lq_get_last_error(b.st) == B.LQ_OK
