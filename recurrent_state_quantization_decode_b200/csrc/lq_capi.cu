@@ -1,6 +1,8 @@
 // C ABI of libleapquant.so (declared in include/leapquant.h): argument
-// validation on the host, then one kernel launch per call.  No call
-// allocates memory or keeps global state.
+// validation on the host, then the call's launches: one kernel, except the
+// host-buffer step (input gather or copies, the decode kernel, the output
+// copy).  No call here allocates memory or keeps global state; the no-alloc
+// variant's fixed staging array lives in lq_noalloc.cu.
 
 #include <cstdint>
 #include <cstring>
