@@ -249,11 +249,14 @@ def cpu_baseline(w: wl.Workload, target_s: float = 15.0) -> dict:
                        f"fp64 C oracle, OpenMP over tiles; {dt:.1f} s of oracle time")}
 
 
+REFERENCE_BUDGET_S = 150.0  # oracle seconds of the whole --impl reference run
+
+
 def reference_arm(args, w: wl.Workload, rank: int, world: int) -> None:
     if rank != 0:
         return
     steps, warm = args.steps, args.warmup
-    budget = 150.0
+    budget = REFERENCE_BUDGET_S
     seqs, windows = oracle_sample_size(w, budget / (steps + warm))
     for _ in range(warm):
         run_oracle_sample(w, seqs, windows)

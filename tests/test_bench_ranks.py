@@ -3,6 +3,7 @@ rank, as torchrun starts them) check the max-over-ranks timing, the whole-job
 rate, the per-rank seeds and that only rank 0 runs and prints the oracle arm.
 The decode path itself shards by sequence and has no collective."""
 import io
+import json
 import os
 import socket
 import sys
@@ -76,3 +77,37 @@ def test_single_rank_needs_no_process_group():
     assert not dist.is_initialized()
     assert bench.max_over_ranks(4.0, 1) == 4.0
     assert bench.whole_job_rate(5, 1, 2, 1000.0) == pytest.approx(10.0)
+
+
+def test_reference_arm_line_keeps_the_contract(monkeypatch):
+    """Rank 0 of --impl reference prints one JSON line with the contract's keys:
+    the oracle timed on host cores, its own e2e with no transfers."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    monkeypatch.setattr(bench, "REFERENCE_BUDGET_S", 0.6)
+
+    class Args:
+        steps, warmup, layers = 2, 1, 8
+
+    out = io.StringIO()
+    with redirect_stdout(out):
+        bench.reference_arm(Args, bench.WORKLOADS["qwen35_9b_gdn"], 0, 1)
+    lines = out.getvalue().strip().splitlines()
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference"
+    assert d["unit"] == bench.UNIT and d["metric"] == bench.METRIC
+    assert d["value"] > 0 and d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1
+    assert d["higher_is_better"] is True and d["vs_baseline"] is None
+    assert d["config"]["workload"] == bench.WORKLOADS["qwen35_9b_gdn"].name
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert cb["sample"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
