@@ -108,3 +108,72 @@ def test_empty_batch_is_a_no_op(B):
 def test_status_strings(B):
     for s in range(8):
         assert B.lq_status_string(s).startswith("LQ_")
+
+
+def _err(B, fn, *args, **kw):
+    with pytest.raises(B.LQError) as ei:
+        fn(*args, **kw)
+    return ei.value.status
+
+
+def test_newer_entry_points_reject_bad_arguments_before_launch(B):
+    """Prefill, checkpoint copies, rollback, the host-buffer step and the
+    timeout test hook: argument errors come back on the host, with no device
+    access (addresses below are never dereferenced)."""
+    cfg = B.make_config(2, 2, 4, 64)
+    good = 1 << 20
+    st = B.lq_state(good, good, good, good, good, good)
+    # prefill: negative length, missing inputs for a non-empty prompt, misaligned S0
+    assert _err(B, B.lq_prefill, cfg, good, good, good, good, good, -1, None, st,
+                stream=0) == B.LQ_ERR_INVALID_ARG
+    assert _err(B, B.lq_prefill, cfg, None, good, good, good, good, 8, None, st,
+                stream=0) == B.LQ_ERR_INVALID_ARG
+    assert _err(B, B.lq_prefill, cfg, good, good, good, good, good, 8, good + 4, st,
+                stream=0) == B.LQ_ERR_MISALIGNED
+    assert _err(B, B.lq_prefill, cfg, good, good, good, good + 2, good, 8, None, st,
+                stream=0) == B.LQ_ERR_MISALIGNED
+    # checkpoint copies: missing slots or pool, negative pool size, misaligned pool
+    for save in (True, False):
+        def call(slots, pool, n):
+            if save:
+                return B.lq_checkpoint_save(cfg, st, slots, pool, n, stream=0)
+            return B.lq_checkpoint_restore(cfg, pool, n, slots, st, stream=0)
+        assert _err(B, call, None, good, 1) == B.LQ_ERR_INVALID_ARG
+        assert _err(B, call, good, None, 1) == B.LQ_ERR_INVALID_ARG
+        assert _err(B, call, good, good, -1) == B.LQ_ERR_INVALID_ARG
+        assert _err(B, call, good, good + 8, 1) == B.LQ_ERR_MISALIGNED
+        assert _err(B, call, good + 2, good, 1) == B.LQ_ERR_MISALIGNED
+    # rollback: missing or misaligned drop counts
+    assert _err(B, B.lq_window_rewind, cfg, st, None, stream=0) == B.LQ_ERR_INVALID_ARG
+    assert _err(B, B.lq_window_rewind, cfg, st, good + 2, stream=0) == B.LQ_ERR_MISALIGNED
+    # host-buffer step: misaligned staging or mask
+    assert _err(B, B.lq_decode_step_host, cfg, good, good, good, good, good, st, good,
+                good + 8, stream=0) == B.LQ_ERR_MISALIGNED
+    assert _err(B, B.lq_decode_step_host, cfg, good, good, good, good, good, st, good, good,
+                active=good + 1, stream=0) == B.LQ_ERR_MISALIGNED
+    # timeout hook: a zero poll limit or an empty batch is refused
+    assert _err(B, B.lq_test_decode_step_timeout, cfg, good, good, good, good, good, st, good,
+                0, stream=0) == B.LQ_ERR_INVALID_ARG
+    empty = B.make_config(0, 2, 4, 64)
+    assert _err(B, B.lq_test_decode_step_timeout, empty, good, good, good, good, good, st,
+                good, 16, stream=0) == B.LQ_ERR_INVALID_ARG
+    # a bad config is reported before anything else
+    bad = B.make_config(2, 2, 4, 96)
+    assert _err(B, B.lq_prefill, bad, good, good, good, good, good, 8, None, st,
+                stream=0) == B.LQ_ERR_UNSUPPORTED
+    assert _err(B, B.lq_window_rewind, bad, st, good, stream=0) == B.LQ_ERR_UNSUPPORTED
+
+
+def test_newer_entry_points_accept_an_empty_batch(B):
+    """batch == 0 returns LQ_OK without touching the device."""
+    cfg = B.make_config(0, 2, 4, 64)
+    good = 1 << 20
+    st = B.lq_state(good, good, good, good, good, good)
+    B.lq_prefill(cfg, good, good, good, good, good, 8, good, st, stream=0)
+    B.lq_prefill(cfg, None, None, None, None, None, 0, None, st, stream=0)
+    B.lq_checkpoint_save(cfg, st, good, good, 4, stream=0)
+    B.lq_checkpoint_restore(cfg, good, 4, good, st, stream=0)
+    B.lq_window_rewind(cfg, st, good, stream=0)
+    B.lq_decode_step_host(cfg, good, good, good, good, good, st, good, good, stream=0)
+    B.lq_decode_step_host_noalloc(cfg, good, good, good, good, good, st, good, stream=0)
+    B.lq_state_init(cfg, good, st, stream=0)
