@@ -111,3 +111,30 @@ def test_reference_arm_line_keeps_the_contract(monkeypatch):
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_clock_sampler_summary_parses_nvidia_smi_lines():
+    """The clocks object of the bench line: median SM clock under load, the max
+    clock, and the throttle reasons seen inside the timed window only."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    cs = bench.ClockSampler(None)
+    na = "Not Active"
+    cs.lines = [
+        (0.5, f"1200, 1965, 300.0, 0x0, {na}, {na}, {na}, {na}"),        # before the window
+        (1.0, f"1965, 1965, 700.0, 0x0, {na}, {na}, {na}, {na}"),
+        (1.1, f"1950, 1965, 990.0, 0x4, {na}, {na}, {na}, Active"),      # power cap
+        (1.2, f"1965, 1965, 800.0, 0x0, {na}, {na}, {na}, {na}"),
+        (1.3, "garbled"),                                                 # skipped
+        (3.0, f"900, 1965, 200.0, 0x8, Active, {na}, {na}, {na}"),       # after the window
+    ]
+    cs.window(0.9, 1.5)
+    s = cs.summary()
+    assert s == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                 "samples": 3}
+    cs.window(0.0, 10.0)
+    s = cs.summary()
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"] and s["samples"] == 5
+    empty = bench.ClockSampler(None)
+    assert empty.summary()["reasons"] == ["no samples"]
