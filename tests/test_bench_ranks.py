@@ -138,3 +138,36 @@ def test_clock_sampler_summary_parses_nvidia_smi_lines():
     assert s["reasons"] == ["hw_slowdown", "sw_power_cap"] and s["samples"] == 5
     empty = bench.ClockSampler(None)
     assert empty.summary()["reasons"] == ["no samples"]
+
+
+def test_algorithmic_bytes_and_profiled_traffic(tmp_path, monkeypatch):
+    """The roofline's numerator: bytes one tile-step must move, item by item
+    (record from the public layout, a half-full window's buffer on average,
+    shared keys split over the value heads of a key head); and the DRAM
+    traffic read from the ncu summary only while the kernel source matches
+    the hash it was captured on."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    w = bench.WORKLOADS["qwen35_9b_gdn"]
+    ab = bench.algorithmic_bytes_per_tile_step(w)
+    d, g = 128, 2
+    record = d * d + 4 * d + 4 * d + 4 * 4 * d + 4 * 4          # codes, sigma, m, lines, ids
+    entry = 4 * d + 4 + 2 * d / g                               # d_s, alpha_s, half a bf16 k_s
+    assert ab == {"record_read": record, "buffer_read": 7.5 * entry, "buffer_append": entry,
+                  "fold_record_write": record / 16, "inputs": 2 * 2 * d / g + 2 * d + 8,
+                  "output": 4 * d, "phase_counter": 8, "total": 27203.0}
+    assert record == 19472
+    assert bench.fp32_bytes_per_tile_step(w) == 2 * 4 * d * d + 520 + 4 * d
+
+    src = tmp_path / "kernel.cu"
+    src.write_text("// kernel v1\n")
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", [str(src)])
+    summary = tmp_path / "summary.md"
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(summary))
+    assert bench.profiled_traffic(10) is None                   # no summary
+    summary.write_text(f"kernel_source_sha: {bench.kernel_source_sha()}\n"
+                       "dram_bytes_per_tile_step: 24911\n")
+    assert bench.profiled_traffic(2048) == 24911 * 2048
+    src.write_text("// kernel v2\n")                            # kernel changed since
+    assert bench.profiled_traffic(2048) is None
