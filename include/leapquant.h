@@ -2,8 +2,9 @@
  * leapquant.h - C ABI of libleapquant.so: the per-token decode step of a
  * Gated DeltaNet (GDN) / Kimi Delta Attention (KDA) layer whose recurrent
  * state is stored in int8, following LeapQuant, with the calls around it:
- * state init, a prefill that ends in the quantizer, partial-window flush,
- * prefix-cache checkpoints, dequantization and the fp32-state comparison
+ * state init, a prefill that ends in the quantizer, the decode step on host
+ * buffers, partial-window flush, prefix-cache checkpoints, speculative
+ * rollback inside a window, dequantization and the fp32-state comparison
  * step.
  *
  * Method sources (page title, section):
@@ -42,8 +43,8 @@
  *  buf_n    [B][Hv] int32 tokens buffered in the current window (0..W-1
  *           between calls).
  *  err      one int32 device error word (bit 0: a corrupt buf_n was seen,
- *           or a checkpoint copy was refused; bit 1: a bounded wait on a
- *           copy expired).
+ *           or a checkpoint copy or a rollback was refused; bit 1: a
+ *           bounded wait on a copy expired).
  * The layout is public: a checkpoint of a tile at a window boundary is a copy
  * of its record.
  *
