@@ -329,6 +329,44 @@ def test_each_technique_reduces_drift():
     assert full < no_comp
 
 
+def _chunked_wy(S, q, k, v, alpha, beta, C, diag_gate):
+    """The recurrence in chunks of C tokens, WY form (numpy, fp64): within a
+    chunk with cumulative gates g_t, the deltas u_t = beta_t (v_t - S_{t-1}
+    D_t k_t) solve (I + A) U = diag(beta) (V - Kg S0^T) with A_ti = beta_t
+    (k_t o g_t) . (k_i / g_i) for i < t; outputs are Qg S0^T + tril(Qg Kh^T) U
+    and the chunk's last state S0 G_C + U^T (Kh o g_C).  An algebraic route
+    independent of the token loop."""
+    out = []
+    for c0 in range(0, len(q), C):
+        Q, K, V, al, be = (x[c0:c0 + C] for x in (q, k, v, alpha, beta))
+        g = np.cumprod(al if diag_gate else al[:, None] * np.ones((1, K.shape[1])), axis=0)
+        Kg, Kh, Qg = K * g, K / g, Q * g
+        A = np.tril(be[:, None] * (Kg @ Kh.T), -1)
+        U = np.linalg.solve(np.eye(len(Q)) + A, be[:, None] * (V - Kg @ S.T))
+        out.append(Qg @ S.T + np.tril(Qg @ Kh.T) @ U)
+        S = S * g[-1][None, :] + U.T @ (Kh * g[-1][None, :])
+    return S, np.concatenate(out)
+
+
+@pytest.mark.parametrize("gate", [0, 1])
+@pytest.mark.parametrize("C", [1, 16, 64])
+def test_exact_recurrence_matches_the_chunked_wy_form(gate, C):
+    rng = np.random.default_rng(40 + gate)
+    dk, dv, T = 16, 12, 100
+    S0 = rng.standard_normal((dv, dk)) * 0.1
+    q = rng.standard_normal((T, dk))
+    k = rng.standard_normal((T, dk))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((T, dv))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal(T)))
+    alpha = (np.exp(-np.logaddexp(0.0, rng.standard_normal((T, dk))) * 0.05) if gate
+             else rng.uniform(0.9, 1.0, T))
+    S_ex, o_ex = exact_run(Cfg(dk, dv, gate=gate), S0, q, k, v, alpha, beta)
+    S_ch, o_ch = _chunked_wy(S0, q, k, v, alpha, beta, C, gate == 1)
+    assert np.max(np.abs(S_ch - S_ex)) < 1e-12
+    assert np.max(np.abs(o_ch - o_ex)) < 1e-12
+
+
 def test_drift_falls_as_the_window_grows():
     """The fixed-state window is what cuts requantization error (zhichai.net
     summary, "Abstract (translated)" item 1): with K = 4 and smoothing 1/2, the
