@@ -474,15 +474,20 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
         ms = max_over_ranks(start.elapsed_time(end), world, device)
         return ms, (sampler.summary() if sample_clocks else None)
 
-    g8 = capture(step_int8)
-    ms8, clocks = timed(g8, args.steps, args.warmup, sample_clocks=True)
+    # NVTX ranges name the bench's phases for a timeline profiler (host-side
+    # push/pop only; the device timing is the CUDA events inside `timed`)
+    nvtx = torch.cuda.nvtx.range
+    with nvtx("int8-state decode: capture, warm-up, timed replay"):
+        g8 = capture(step_int8)
+        ms8, clocks = timed(g8, args.steps, args.warmup, sample_clocks=True)
     err = max(B.lq_get_last_error(ly.ds.st, stream.cuda_stream) for ly in layers)
     if err != B.LQ_OK:
         raise RuntimeError(f"device error word set: {B.lq_status_string(err)}")
     del g8
-    g32 = capture(step_fp32)
     steps32 = max(3, args.steps // 4)
-    ms32, _ = timed(g32, steps32, args.warmup)
+    with nvtx("fp32-state decode: capture, warm-up, timed replay"):
+        g32 = capture(step_fp32)
+        ms32, _ = timed(g32, steps32, args.warmup)
     del g32
 
     units_per_step = w.tiles * W * L               # per rank
@@ -543,8 +548,9 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
         start.record(stream)
         for st2 in streams[1:]:
             st2.wait_event(start)
-        for _ in range(e2e_steps):
-            step_host()
+        with nvtx("end to end through lq_decode_step_host, timed"):
+            for _ in range(e2e_steps):
+                step_host()
         for st2 in streams[1:]:
             done = torch.cuda.Event()
             done.record(st2)
@@ -562,7 +568,8 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
     # prefill of one layer's tiles over a prompt, ending in the quantizer
     prefill = None
     if not args.no_prefill:
-        prefill = prefill_measure(B, w, layers[0], stream, device, world)
+        with nvtx("prefill of one layer"):
+            prefill = prefill_measure(B, w, layers[0], stream, device, world)
 
     if rank != 0:
         return
@@ -591,7 +598,8 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
     if prefill is not None:
         line["prefill"] = prefill
     if world == 1 and not args.no_cpu:
-        line["cpu_baseline"] = cpu_baseline(w)
+        with nvtx("CPU oracle baseline"):
+            line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
 
 
