@@ -279,7 +279,36 @@ def reference_arm(args, w: wl.Workload, rank: int, world: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+L2_BYTES = 126 * 2**20  # B200 L2
+
+
+def working_set_bytes(w: wl.Workload, layers: int) -> int:
+    """Device bytes one timed int8 step touches: every layer's records, window
+    buffers and counters, the W tokens of inputs it decodes and its output."""
+    d, W, tiles = w.d, w.window, w.tiles
+    inb = 2 if w.io_bf16 else 4
+    ga = d if w.gate == wl.GATE_DIAG else 1
+    record = (d * d + 8 * d + 4 * w.n_comp * d + 4 * w.n_comp + 15) // 16 * 16
+    state = (tiles * record + w.batch * w.num_k_heads * W * d * inb + tiles * W * d * 4
+             + tiles * (W * d * 4 if ga > 1 else 16 * 4) + tiles * 4)
+    inputs = W * (2 * w.batch * w.num_k_heads * d * inb + tiles * d * inb
+                  + tiles * ga * 4 + tiles * 4)
+    return layers * (state + inputs + tiles * d * 4)
+
+
+def l2_statement(ws: int) -> str:
+    mb, l2 = ws / 2**20, L2_BYTES / 2**20
+    if ws < L2_BYTES:
+        return (f"working set {mb:.0f} MB fits in the {l2:.0f} MB L2: L2-resident, "
+                "not an HBM figure")
+    if ws < 2 * L2_BYTES:
+        return f"working set {mb:.0f} MB, under twice the {l2:.0f} MB L2: partly L2-resident"
+    return (f"inputs larger than L2: working set {mb:.0f} MB = {ws / L2_BYTES:.1f}x the "
+            f"{l2:.0f} MB L2 (layer states cycled every token)")
+
+
 def workload_config(w: wl.Workload, layers: int) -> dict:
+    ws = working_set_bytes(w, layers)
     return {"workload": w.name, "batch": w.batch, "num_k_heads": w.num_k_heads,
             "num_v_heads": w.num_v_heads, "d_k": w.d, "d_v": w.d,
             "gate": "scalar (GDN)" if w.gate == wl.GATE_SCALAR else "diagonal (KDA)",
@@ -287,7 +316,8 @@ def workload_config(w: wl.Workload, layers: int) -> dict:
             "compensators": w.n_comp, "smooth": w.smooth, "layers_cycled": layers,
             "tiles_per_layer": w.tiles,
             "step": f"one {w.window}-token window x {layers} layers",
-            "l2": "inputs larger than L2 (layer states cycled every token)"}
+            "working_set_mb": round(ws / 2**20, 1),
+            "l2": l2_statement(ws)}
 
 
 # ---------------------------------------------------------------------------

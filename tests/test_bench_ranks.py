@@ -171,3 +171,28 @@ def test_algorithmic_bytes_and_profiled_traffic(tmp_path, monkeypatch):
     assert bench.profiled_traffic(2048) == 24911 * 2048
     src.write_text("// kernel v2\n")                            # kernel changed since
     assert bench.profiled_traffic(2048) is None
+
+
+def test_working_set_and_l2_statement():
+    """The config's L2 statement: the step's working set (every layer's state
+    per the C library's layout, its W tokens of inputs and its output) decides
+    whether a run streams from HBM or sits in the 126 MB L2."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from recurrent_state_quantization_decode_b200 import binding as B
+
+    for name in ("qwen35_9b_gdn", "kimi_linear_kda", "gdn_sweep_b8"):
+        w = bench.WORKLOADS[name]
+        L = B.lq_state_layout(B.config_for(w))
+        state = (L.records_bytes + L.buf_k_bytes + L.buf_d_bytes + L.buf_g_bytes
+                 + L.buf_n_bytes)
+        inb = 2 if w.io_bf16 else 4
+        ga = w.d if w.gate == 1 else 1
+        inputs = w.window * (2 * w.batch * w.num_k_heads * w.d * inb
+                             + w.tiles * w.d * inb + w.tiles * ga * 4 + w.tiles * 4)
+        out = w.tiles * w.d * 4
+        assert bench.working_set_bytes(w, 8) == 8 * (state + inputs + out), name
+    big = bench.workload_config(bench.WORKLOADS["qwen35_9b_gdn"], 8)
+    assert big["l2"].startswith("inputs larger than L2") and big["working_set_mb"] > 2 * 126
+    small = bench.workload_config(bench.WORKLOADS["gdn_sweep_b8"], 8)
+    assert "L2-resident" in small["l2"] and small["working_set_mb"] < 126
