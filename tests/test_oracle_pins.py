@@ -204,6 +204,40 @@ def test_quantize_column_and_row_scaling_invariance():
     np.testing.assert_array_equal(r0.sig.astype(np.float64) * 2.0 ** f, r1.sig)
 
 
+def test_half_smoothing_takes_the_square_root_of_the_column_max():
+    """Default smoothing (exponent 1/2), pinned by exact values.  Every column
+    of S holds one entry of magnitude exactly 1 and the rest below it, so its
+    max is 1.  Scaling column j by 4^e_j makes that max 4^e_j, whose square
+    root is exactly 2^e_j: m_j must be 2^e_j (an exponent of 1/4 or 1 would
+    give 2^(e_j/2) or 4^e_j), and the smoothed residual S_ij 4^e_j / 2^e_j =
+    S_ij 2^e_j must quantize exactly as S diag(2^e) does with smoothing off
+    (which would fail if the kernel multiplied by m instead of dividing)."""
+    rng = np.random.default_rng(12)
+    dk, dv = 24, 20
+    S = rng.uniform(-0.99, 0.99, (dv, dk)).astype(np.float32).astype(np.float64)
+    rows = rng.integers(0, dv, dk)
+    S[rows, np.arange(dk)] = rng.choice([-1.0, 1.0], dk)
+    e = rng.integers(-5, 6, dk).astype(np.float64)
+    e[:2] = (3.0, -3.0)                       # odd exponents: 2^(e/2) is not a power of two
+    half = quantize(Cfg(dk, dv, K=0, smooth=0.5), S * 4.0 ** e[None, :])
+    np.testing.assert_array_equal(half.m.astype(np.float64), 2.0 ** e)
+    off = quantize(Cfg(dk, dv, K=0, smooth=0.0), S * 2.0 ** e[None, :])
+    np.testing.assert_array_equal(half.Q, off.Q)
+    np.testing.assert_array_equal(half.sig, off.sig)
+
+
+def test_codes_round_half_to_even():
+    """A constructed exact tie: smoothing off and one row whose max is 127, so
+    its scale is 127/127 = 1 and every code is rint of the entry itself.
+    Entries k + 1/2 must go to the even neighbour (0.5 -> 0, 2.5 -> 2,
+    -2.5 -> -2, 126.5 -> 126, 1.5 -> 2, -3.5 -> -4); rounding half away from
+    zero would give 1, 3, -3, 127, 2, -4."""
+    row = np.array([127.0, 0.5, 2.5, -2.5, 126.5, 1.5, -3.5, -0.5])
+    rec = quantize(Cfg(8, 1, K=0, smooth=0.0), row[None, :])
+    assert rec.sig[0] == np.float32(1.0)
+    assert list(rec.Q[0]) == [127, 0, 2, -2, 126, 2, -4, 0]
+
+
 def test_smoothing_reduces_error_on_column_outliers():
     rng = np.random.default_rng(9)
     dk = dv = 64
