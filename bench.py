@@ -1,7 +1,8 @@
 """Benchmark of the int8-state LeapQuant GDN/KDA decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload qwen35_9b_gdn|kimi_linear_kda|gdn_sweep_bB] [--layers L]
+                    [--workload kimi_linear_kda|qwen35_9b_gdn|gdn_sweep_bB|ragged_gdn]
+                    [--layers L] [--no-others]
 
 One step = one 16-token quantization window (15 plain decode tokens and the
 boundary token whose kernel also folds, compensates, smooths and requantizes)
@@ -11,7 +12,13 @@ above the 126 MB L2, so every step streams its state from HBM.
 
 value = tile-steps/s (one tile-step = one decode token of one value head of
 one layer) with all inputs resident in HBM, timed with CUDA events around a
-CUDA-graph replay of K steps.  The same line carries: the in-house fp32-state
+CUDA-graph replay of K steps.  The default workload is the Kimi-Linear-like
+KDA layer (128 sequences x 32 heads = 4,096 tiles, the batch x heads >= 4096
+regime); the line also carries, as sub-objects with their own fp32-state
+comparison and roofline, the Qwen3.5-9B-like GDN layer (2,048 tiles), the
+largest bandwidth-sweep point (32,768 tiles) and a ragged batch whose
+sequences sit in different window phases (8,192 tiles, about 1/16 of them
+folding at every token).  The same line carries: the in-house fp32-state
 kernel on the same workload and its speedup ratio, the roofline of the decode
 kernel against the measured HBM copy bandwidth, end-to-end throughput through
 the host-buffer C entry point, the CPU oracle timed on a sample, and the SM
@@ -48,8 +55,13 @@ METRIC = ("decode tokens/s·head (int8 state) & achieved HBM GB/s vs 8 TB/s; "
 UNIT = "tile-steps/s"
 NOMINAL_HBM_GBS = 8000.0
 WORKLOADS = {"qwen35_9b_gdn": wl.QWEN35_9B_GDN, "kimi_linear_kda": wl.KIMI_LINEAR_KDA,
+             "ragged_gdn": wl.RAGGED,
              **{f"gdn_sweep_b{b}": wl.sweep_workload(b) for b in wl.SWEEP_BATCHES}}
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_qwen35_9b_gdn.md")
+DEFAULT_WORKLOAD = "kimi_linear_kda"
+# the other workloads the default line reports as sub-objects, with the layer
+# count each cycles (enough to keep the working set above L2)
+OTHER_WORKLOADS = (("qwen35_9b_gdn", 8), ("gdn_sweep_b1024", 2), ("ragged_gdn", 4))
+PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = [os.path.join(ROOT, "recurrent_state_quantization_decode_b200", "csrc", f)
                   for f in ("lq_decode.cu", "lq_internal.h")]
 
@@ -98,12 +110,22 @@ def kernel_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(tiles: int):
-    """DRAM bytes per launch of the decode kernel from the committed ncu summary,
-    scaled to `tiles`; None if the summary is missing or the kernel source has
-    changed since it was captured."""
+def profile_summary_path(key: str) -> str:
+    """The committed ncu summary of the decode kernel on workload `key`."""
+    return os.path.join(PROFILE_DIR, f"decode_kernel_{key}.md")
+
+
+def kernel_label(w: wl.Workload) -> str:
+    return (f"decode_kernel<{w.d},{'bf16' if w.io_bf16 else 'f32'},"
+            f"{'KDA' if w.gate == wl.GATE_DIAG else 'GDN'}> (int8 state)")
+
+
+def profiled_traffic(tiles: int, key: str = "qwen35_9b_gdn"):
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary
+    of workload `key`, scaled to `tiles`; None if the summary is missing or the
+    kernel source has changed since it was captured."""
     try:
-        txt = open(PROFILE_SUMMARY).read()
+        txt = open(profile_summary_path(key)).read()
     except OSError:
         return None
     sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
@@ -324,19 +346,27 @@ def workload_config(w: wl.Workload, layers: int) -> dict:
 # GPU arm
 # ---------------------------------------------------------------------------
 
-class Layer:
-    """One layer's stored state, fp32 comparison state and W tokens of inputs."""
+STATE_POOL = 512  # distinct initial states drawn per layer; larger batches repeat them
 
-    def __init__(self, B, w: wl.Workload, seed: int, device):
+
+class Layer:
+    """One layer's stored state, fp32 comparison state and W tokens of inputs.
+    With `phases`, sequence b first decodes phases[b] tokens (active masks), so
+    that the layer's tiles sit in different window phases."""
+
+    def __init__(self, B, w: wl.Workload, seed: int, device, phases=None):
         import torch
 
         rng = np.random.default_rng(seed)
-        S0, _, _ = wl.initial_states(rng, w.tiles, w.d, w.d)
+        pool = min(w.tiles, STATE_POOL)
+        S0, _, _ = wl.initial_states(rng, pool, w.d, w.d)
         ti = wl.token_inputs(rng, w, w.window)
         dt = torch.bfloat16 if w.io_bf16 else torch.float32
         self.cfg = B.config_for(w)
         self.ds = B.DeviceState(self.cfg, device=device)
         S0_dev = torch.from_numpy(S0).to(device)
+        if pool < w.tiles:
+            S0_dev = S0_dev[torch.arange(w.tiles, device=device) % pool].contiguous()
         B.lq_state_init(self.cfg, S0_dev, self.ds.st)
         self.S32 = S0_dev  # the fp32-state path starts from the same states
         self.q = torch.from_numpy(ti.q).to(device=device, dtype=dt)
@@ -346,6 +376,13 @@ class Layer:
         self.beta = torch.from_numpy(ti.beta).to(device)
         self.out = torch.empty((w.batch, w.num_v_heads, w.d), dtype=torch.float32, device=device)
         self.host = None
+        if phases is not None:
+            ph = torch.as_tensor(phases, dtype=torch.int32, device=device)
+            for t in range(int(ph.max().item())):
+                act = (ph > t).to(torch.int32)
+                B.lq_decode_step(self.cfg, self.q[t], self.k[t], self.v[t], self.alpha[t],
+                                 self.beta[t], self.ds.st, self.out, active=act)
+            torch.cuda.synchronize(device)
 
     def pin_host_inputs(self):
         import torch
@@ -355,6 +392,13 @@ class Layer:
         self.host_out = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
         self.staging = torch.empty(self.ds.layout.host_staging_bytes, dtype=torch.uint8,
                                    device=self.out.device)
+
+
+def ragged_phases(w: wl.Workload, seed: int) -> np.ndarray:
+    """Per-sequence window phases of the ragged workload (its recipe's phase
+    offsets): sequence b has decoded phase[b] tokens of its current window."""
+    _, phase = wl.ragged_lengths(np.random.default_rng(seed), w.batch)
+    return phase
 
 
 # ---------------------------------------------------------------------------
@@ -429,17 +473,29 @@ def prefill_measure(B, w: wl.Workload, ly, stream, device, world: int) -> dict:
             "kernel": "prefill_kernel (exact recurrence, state on chip, then quantizer)"}
 
 
-def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> None:
+def load_peaks() -> tuple[float, str]:
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        peaks = {}
+    if "hbm_gbs" in peaks:
+        return float(peaks["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def measure_decode(B, w: wl.Workload, key: str, L: int, steps: int, warmup: int, stream,
+                   device, world: int, rank: int, sample_clocks: bool = False,
+                   phases: bool = False, keep_layers: bool = False) -> dict:
+    """Time `steps` steps (one W-token window for every tile of L layers) of
+    the int8-state decode and steps/4 of the fp32-state kernel, each as a
+    CUDA-graph replay after `warmup` replays; return the workload's figures."""
     import torch
     import torch.distributed as dist
 
-    from recurrent_state_quantization_decode_b200 import binding as B
-
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    L = args.layers
-    layers = [Layer(B, w, seed=layer_seed(rank, l), device=device) for l in range(L)]
-    stream = torch.cuda.Stream(device=device)
+    layers = []
+    for l in range(L):
+        ph = ragged_phases(w, layer_seed(rank, l)) if phases else None
+        layers.append(Layer(B, w, seed=layer_seed(rank, l), device=device, phases=ph))
     W = w.window
     launches_per_step = W * L
 
@@ -469,7 +525,7 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
         if world > 1:
             dist.barrier()
 
-    def timed(graph, steps, warmup, sample_clocks=False):
+    def timed(graph, n, sample):
         with torch.cuda.stream(stream):
             for _ in range(warmup):
                 graph.replay()
@@ -483,63 +539,105 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
             uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
         except Exception:
             pass
-        sampler = ClockSampler(uuid if sample_clocks else None)
-        if sample_clocks:
+        sampler = ClockSampler(uuid if sample else None)
+        if sample:
             sampler.__enter__()
             time.sleep(0.3)
         wall0 = time.time()
         with torch.cuda.stream(stream):
             start.record(stream)
-            for _ in range(steps):
+            for _ in range(n):
                 graph.replay()
             end.record(stream)
         torch.cuda.synchronize()
         wall1 = time.time()
-        if sample_clocks:
+        if sample:
             time.sleep(0.15)
             sampler.__exit__(None, None, None)
             sampler.window(wall0, wall1)
         barrier()
         torch.cuda.synchronize()
         ms = max_over_ranks(start.elapsed_time(end), world, device)
-        return ms, (sampler.summary() if sample_clocks else None)
+        return ms, (sampler.summary() if sample else None)
 
-    # NVTX ranges name the bench's phases for a timeline profiler (host-side
-    # push/pop only; the device timing is the CUDA events inside `timed`)
     nvtx = torch.cuda.nvtx.range
-    with nvtx("int8-state decode: capture, warm-up, timed replay"):
+    with nvtx(f"int8-state decode ({key}): capture, warm-up, timed replay"):
         g8 = capture(step_int8)
-        ms8, clocks = timed(g8, args.steps, args.warmup, sample_clocks=True)
+        ms8, clocks = timed(g8, steps, sample_clocks)
     err = max(B.lq_get_last_error(ly.ds.st, stream.cuda_stream) for ly in layers)
     if err != B.LQ_OK:
         raise RuntimeError(f"device error word set: {B.lq_status_string(err)}")
     del g8
-    steps32 = max(3, args.steps // 4)
-    with nvtx("fp32-state decode: capture, warm-up, timed replay"):
+    steps32 = max(3, steps // 4)
+    with nvtx(f"fp32-state decode ({key}): capture, warm-up, timed replay"):
         g32 = capture(step_fp32)
-        ms32, _ = timed(g32, steps32, args.warmup)
+        ms32, _ = timed(g32, steps32, False)
     del g32
 
     units_per_step = w.tiles * W * L               # per rank
-    value = whole_job_rate(units_per_step, world, args.steps, ms8)
+    value = whole_job_rate(units_per_step, world, steps, ms8)
     value32 = whole_job_rate(units_per_step, world, steps32, ms32)
-    ms_per_step = ms8 / args.steps
-
     # roofline of the decode kernel (algorithmic bytes / graph time per launch)
     ab = algorithmic_bytes_per_tile_step(w)
     bytes_per_launch = ab["total"] * w.tiles
-    launch_s = (ms8 / 1e3) / (args.steps * launches_per_step)
+    launch_s = (ms8 / 1e3) / (steps * launches_per_step)
     achieved = bytes_per_launch / launch_s / 1e9
-    peaks = {}
-    try:
-        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-    except (OSError, ValueError):
-        pass
-    peak = float(peaks.get("hbm_gbs", 6650.0))
-    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
-    traffic = profiled_traffic(w.tiles)
+    peak, peak_src = load_peaks()
     fp32_bytes = fp32_bytes_per_tile_step(w) * w.tiles
     fp32_achieved = fp32_bytes / ((ms32 / 1e3) / (steps32 * launches_per_step)) / 1e9
+    cfg = workload_config(w, L)
+    if w.tiles > STATE_POOL:
+        cfg["initial_states"] = f"{STATE_POOL} drawn per layer, repeated over the tiles"
+    if phases:
+        cfg["window_phases"] = ("per sequence, the recipe's offsets U{0..15}: about 1/16 "
+                                "of the tiles fold at every token")
+    res = {
+        "workload": w.name, "value": value, "unit": UNIT, "steps": steps,
+        "ms_per_step": ms8 / steps, "config": cfg,
+        "gpu_launches": steps * launches_per_step,
+        "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
+        "bytes_per_value": {"stored": ab["record_read"] / (w.d * w.d),
+                            "moved_per_step": ab["total"] / (w.d * w.d)},
+        "fp32_state": {"value": value32, "unit": UNIT, "ms_per_step": ms32 / steps32,
+                       "hbm_gbs": fp32_achieved, "steps": steps32,
+                       "kernel": f"fp32_step_kernel<{w.d}> (fp32 state)"},
+        "speedup_vs_fp32_state": value / value32,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(w.tiles, key),
+                     "peak_source": peak_src, "kernel": kernel_label(w),
+                     "algorithmic_bytes_per_tile_step": ab["total"],
+                     "launch_time": ("graph replay time / launches (includes inter-kernel "
+                                     "gaps)")},
+    }
+    if clocks is not None:
+        res["clocks"] = clocks
+    if keep_layers:
+        res["_layers"] = layers
+    return res
+
+
+def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+
+    from recurrent_state_quantization_decode_b200 import binding as B
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    L = args.layers
+    stream = torch.cuda.Stream(device=device)
+    nvtx = torch.cuda.nvtx.range
+    W = w.window
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    main = measure_decode(B, w, args.workload, L, args.steps, args.warmup, stream, device,
+                          world, rank, sample_clocks=True,
+                          phases=args.workload == "ragged_gdn", keep_layers=True)
+    layers = main.pop("_layers")
+    units_per_step = w.tiles * W * L               # per rank
 
     # end to end through the host-buffer entry point (pinned host memory)
     e2e = None
@@ -554,9 +652,7 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
         # Four streams, layer index mod 4 picks one (fewer when L is not a
         # multiple): each layer stays on its own stream (its tokens in order,
         # its own staging and output buffers), while one layer's input gather
-        # and output copy overlap other layers' kernels.  With the gather
-        # kernel, four streams measured 41.7 M tile-steps/s against 36.5 M
-        # for two.
+        # and output copy overlap other layers' kernels.
         n_streams = 4 if L % 4 == 0 else (2 if L % 2 == 0 else 1)
         streams = [stream] + [torch.cuda.Stream(device=device) for _ in range(n_streams - 1)]
 
@@ -600,33 +696,43 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
     if not args.no_prefill:
         with nvtx("prefill of one layer"):
             prefill = prefill_measure(B, w, layers[0], stream, device, world)
+    del layers
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    # the other workloads, each with its own fp32 comparison and roofline
+    others = {}
+    if not args.no_others and args.workload == DEFAULT_WORKLOAD:
+        sub_steps = max(5, args.steps // 5)
+        for key, lay in OTHER_WORKLOADS:
+            with nvtx(f"sub-workload {key}"):
+                others[key] = measure_decode(B, WORKLOADS[key], key, lay, sub_steps,
+                                             args.warmup, stream, device, world, rank,
+                                             phases=key == "ragged_gdn")
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
 
     if rank != 0:
         return
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "metric": METRIC, "value": main["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "state_dtype": "int8", "data": "synthetic", "config": workload_config(w, L),
-        "gpu_launches": args.steps * launches_per_step,
-        "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
-        "bytes_per_value": {"stored": ab["record_read"] / (w.d * w.d),
-                            "moved_per_step": ab["total"] / (w.d * w.d)},
-        "fp32_state": {"value": value32, "unit": UNIT, "ms_per_step": ms32 / steps32,
-                       "hbm_gbs": fp32_achieved, "steps": steps32},
-        "speedup_vs_fp32_state": value / value32,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": peak_src,
-                     "kernel": "decode_kernel<128,bf16,GDN> (int8 state)",
-                     "algorithmic_bytes_per_tile_step": ab["total"],
-                     "launch_time": "graph replay time / launches (includes inter-kernel gaps)"},
-        "clocks": clocks,
+        "state_dtype": "int8", "data": "synthetic", "config": main["config"],
+        "gpu_launches": main["gpu_launches"],
+        "hbm_gbs": main["hbm_gbs"], "hbm_frac_of_8tbs": main["hbm_frac_of_8tbs"],
+        "bytes_per_value": main["bytes_per_value"],
+        "fp32_state": main["fp32_state"],
+        "speedup_vs_fp32_state": main["speedup_vs_fp32_state"],
+        "roofline": main["roofline"],
+        "clocks": main.get("clocks"),
     }
     if e2e is not None:
         line["e2e"] = e2e
     if prefill is not None:
         line["prefill"] = prefill
+    if others:
+        line["other_workloads"] = others
     if world == 1 and not args.no_cpu:
         with nvtx("CPU oracle baseline"):
             line["cpu_baseline"] = cpu_baseline(w)
@@ -639,11 +745,13 @@ def main() -> None:
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen35_9b_gdn")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the other workloads' sub-objects of the default line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -191,7 +191,10 @@ lq_status lq_decode_step(const lq_config *cfg, const void *q, const void *k, con
  * 16-byte aligned), runs the step, and copies o back to out_host, all
  * asynchronously on `stream` (the caller synchronizes before reading
  * out_host).  The state stays on the device.  active is a device pointer, as
- * above.
+ * above; with it, rows of inactive sequences in out_host come back unchanged
+ * (the call reads out_host's current rows into the staging before the step and
+ * copies the whole output region back), so out_host must stay unchanged by
+ * the host until the stream reaches the output copy.
  *  - Inputs in pinned memory that the device maps at the same address
  *    (cudaHostAlloc / cudaMallocHost memory under unified addressing, as the
  *    driver reports through cudaPointerGetAttributes for both ends of the
@@ -219,13 +222,18 @@ lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const vo
  *  - Problems whose staging (layout.host_staging_bytes) exceeds
  *    LQ_NOALLOC_STAGING_MAX_BYTES are rejected with LQ_ERR_TOO_LARGE before
  *    anything is launched.
- *  - All calls share the array and it keeps the previous call's contents; the
- *    output region is cleared on every call, so outputs of inactive sequences
- *    read back as zeros.  Calls that overlap on the GPU (other streams or other
- *    threads) race on the array: the caller must order them.
+ *  - Every argument is checked, as lq_decode_step_host checks it, before the
+ *    array is looked up or touched.
+ *  - All calls share the array and it keeps the previous call's contents.  No
+ *    stale byte reaches the caller: every output row copied back is written
+ *    by this call (with an active mask, inactive rows come back unchanged, as
+ *    for lq_decode_step_host).  Calls that overlap on the GPU (other streams
+ *    or other threads) race on the array: the caller must order them.
  *  - The first call on each device looks up the array's device address (with
  *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *    stream capture.  The cached address belongs to the device's primary
+ *    context: after cudaDeviceReset, reload the library before calling this
+ *    entry point again on that device.
  * Arguments and results are otherwise those of lq_decode_step_host. */
 #define LQ_NOALLOC_STAGING_MAX_BYTES ((size_t)8 << 20)
 lq_status lq_decode_step_host_noalloc(const lq_config *cfg, const void *q_host,

@@ -20,7 +20,7 @@ LIB = os.path.join(PKG, "libleapquant.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("lq_decode.cu", "lq_fp32.cu", "lq_checkpoint.cu",
                                             "lq_hostio.cu", "lq_capi.cu", "lq_noalloc.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, h) for h in ("lq_internal.h", "lq_checkpoint.h",
-                                                          "lq_hostio.h")] + \
+                                                          "lq_hostio.h", "lq_capi_internal.h")] + \
     [os.path.join(INCLUDE, "leapquant.h")]
 
 

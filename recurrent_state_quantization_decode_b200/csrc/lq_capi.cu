@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/leapquant.h"
+#include "lq_capi_internal.h"
 #include "lq_checkpoint.h"
 #include "lq_hostio.h"
 #include "lq_internal.h"
@@ -23,7 +24,6 @@ bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p
 
 size_t in_size(const lq_config *c) { return c->in_dtype == LQ_DTYPE_BF16 ? 2 : 4; }
 size_t out_size(const lq_config *c) { return c->out_dtype == LQ_DTYPE_BF16 ? 2 : 4; }
-size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Shape and option checks shared by every entry point.
 lq_status check_config(const lq_config *c) {
@@ -95,7 +95,32 @@ KParams make_params(const lq_config *c, const lq_state *st) {
 
 lq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LQ_OK : LQ_ERR_CUDA; }
 
+lq::StagingLayout staging_of(const lq_config *c) {
+  return lq::staging_layout(c->batch, c->num_k_heads, c->num_v_heads, c->d, in_size(c),
+                            out_size(c), c->gate == LQ_GATE_DIAG);
+}
+
 }  // namespace
+
+namespace lq {
+
+// Every argument check of the host-buffer step except its staging pointer, so
+// that the no-alloc variant rejects a bad call before it touches its array.
+lq_status check_host_step(const lq_config *cfg, const void *q_host, const void *k_host,
+                          const void *v_host, const float *alpha_host, const float *beta_host,
+                          const lq_state *st, const void *out_host, const int32_t *active) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if ((s = check_io(cfg, q_host, k_host, v_host, alpha_host, beta_host, out_host)) != LQ_OK)
+    return s;
+  if (!aligned_to(active, 4)) return LQ_ERR_MISALIGNED;
+  return LQ_OK;
+}
+
+size_t host_staging_bytes(const lq_config *cfg) { return staging_of(cfg).total; }
+
+}  // namespace lq
 
 extern "C" {
 
@@ -123,7 +148,6 @@ lq_status lq_state_layout(const lq_config *cfg, lq_layout *out) {
   const lq::RecLayout L = lq::record_layout(cfg->d, cfg->n_comp);
   const size_t B = cfg->batch, Hk = cfg->num_k_heads, Hv = cfg->num_v_heads;
   const size_t d = cfg->d, W = cfg->window, tiles = B * Hv;
-  const size_t ga = cfg->gate == LQ_GATE_DIAG ? d : 1;
   out->record_bytes = L.bytes;
   out->off_sigma = L.off_sig;
   out->off_m = L.off_m;
@@ -136,9 +160,7 @@ lq_status lq_state_layout(const lq_config *cfg, lq_layout *out) {
   out->buf_n_bytes = tiles * 4;
   out->err_bytes = 4;
   out->fp32_state_bytes = tiles * d * d * 4;
-  out->host_staging_bytes = 2 * round256(B * Hk * d * in_size(cfg)) +
-                            round256(tiles * d * in_size(cfg)) + round256(tiles * ga * 4) +
-                            round256(tiles * 4) + round256(tiles * d * out_size(cfg));
+  out->host_staging_bytes = staging_of(cfg).total;
   return LQ_OK;
 }
 
@@ -276,33 +298,28 @@ lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const vo
                               const void *v_host, const float *alpha_host,
                               const float *beta_host, const lq_state *st, void *out_host,
                               void *staging, const int32_t *active, void *stream) {
-  lq_status s = check_config(cfg);
+  lq_status s =
+      lq::check_host_step(cfg, q_host, k_host, v_host, alpha_host, beta_host, st, out_host, active);
   if (s != LQ_OK) return s;
-  if ((s = check_state(cfg, st)) != LQ_OK) return s;
-  if ((s = check_io(cfg, q_host, k_host, v_host, alpha_host, beta_host, out_host)) != LQ_OK)
-    return s;
   if (staging == nullptr) return LQ_ERR_INVALID_ARG;
-  if (!aligned16(staging) || !aligned_to(active, 4)) return LQ_ERR_MISALIGNED;
+  if (!aligned16(staging)) return LQ_ERR_MISALIGNED;
   if (cfg->batch == 0) return LQ_OK;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const size_t B = cfg->batch, Hk = cfg->num_k_heads, Hv = cfg->num_v_heads, d = cfg->d;
-  const size_t tiles = B * Hv, ga = cfg->gate == LQ_GATE_DIAG ? d : 1;
-  const size_t nq = B * Hk * d * in_size(cfg), nv = tiles * d * in_size(cfg);
-  const size_t na = tiles * ga * 4, nb = tiles * 4, no = tiles * d * out_size(cfg);
+  const lq::StagingLayout sl = staging_of(cfg);
   uint8_t *base = static_cast<uint8_t *>(staging);
-  uint8_t *dq = base;
-  uint8_t *dk = dq + round256(nq);
-  uint8_t *dv = dk + round256(nq);
-  uint8_t *da = dv + round256(nv);
-  uint8_t *db = da + round256(na);
-  uint8_t *dout = db + round256(nb);
+  uint8_t *dout = base + sl.out;
   // Inputs in device-mapped pinned memory are read by one gather kernel over
-  // the host link; any other host memory goes through the copy engine.
-  const void *src[5] = {q_host, k_host, v_host, alpha_host, beta_host};
-  void *dst[5] = {dq, dk, dv, da, db};
-  const size_t bytes[5] = {nq, nq, nv, na, nb};
+  // the host link; any other host memory goes through the copy engine.  With
+  // an active mask the kernel writes only active sequences' rows, and the
+  // whole output region is copied back: the host's current output rows go
+  // into the staging first, so that inactive sequences read back unchanged.
+  const void *src[6] = {q_host, k_host, v_host, alpha_host, beta_host, out_host};
+  void *dst[6] = {base + sl.q, base + sl.k, base + sl.v, base + sl.alpha, base + sl.beta, dout};
+  const size_t bytes[6] = {sl.q_bytes, sl.q_bytes, sl.v_bytes, sl.alpha_bytes, sl.beta_bytes,
+                           sl.out_bytes};
+  const int nsrc = active != nullptr ? 6 : 5;
   lq::GatherList gather{};
-  for (int i = 0; i < 5; ++i) {
+  for (int i = 0; i < nsrc; ++i) {
     if (const void *view = lq::device_view_of_host(src[i], bytes[i])) {
       gather.seg[gather.n++] = lq::GatherSeg{view, dst[i], bytes[i]};
     } else if (cudaMemcpyAsync(dst[i], src[i], bytes[i], cudaMemcpyHostToDevice, cs) !=
@@ -312,15 +329,15 @@ lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const vo
   }
   if (lq::launch_gather(gather, cs) != cudaSuccess) return LQ_ERR_CUDA;
   KParams p = make_params(cfg, st);
-  p.q = dq;
-  p.k = dk;
-  p.v = dv;
-  p.alpha = reinterpret_cast<const float *>(da);
-  p.beta = reinterpret_cast<const float *>(db);
+  p.q = base + sl.q;
+  p.k = base + sl.k;
+  p.v = base + sl.v;
+  p.alpha = reinterpret_cast<const float *>(base + sl.alpha);
+  p.beta = reinterpret_cast<const float *>(base + sl.beta);
   p.out = dout;
   p.mask = active;
   if (lq::launch_decode(p, cs) != cudaSuccess) return LQ_ERR_CUDA;
-  if (cudaMemcpyAsync(out_host, dout, no, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+  if (cudaMemcpyAsync(out_host, dout, sl.out_bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
     return LQ_ERR_CUDA;
   return LQ_OK;
 }

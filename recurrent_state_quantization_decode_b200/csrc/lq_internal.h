@@ -52,6 +52,37 @@ struct KParams {
 
 constexpr uint32_t kWaitLimitDefault = 1u << 24;
 
+// Device staging of the host-buffer decode step: q, k, v, alpha, beta and the
+// output, each at a 256-byte aligned offset.  The one definition of this
+// layout, used by lq_state_layout (its size), lq_decode_step_host and the
+// no-alloc variant.
+struct StagingLayout {
+  size_t q, k, v, alpha, beta, out;  // byte offsets
+  size_t q_bytes, v_bytes, alpha_bytes, beta_bytes, out_bytes;
+  size_t total;
+};
+
+inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+inline StagingLayout staging_layout(size_t B, size_t Hk, size_t Hv, size_t d, size_t in_bytes,
+                                    size_t out_bytes, bool gate_diag) {
+  StagingLayout s;
+  const size_t tiles = B * Hv;
+  s.q_bytes = B * Hk * d * in_bytes;
+  s.v_bytes = tiles * d * in_bytes;
+  s.alpha_bytes = tiles * (gate_diag ? d : 1) * 4;
+  s.beta_bytes = tiles * 4;
+  s.out_bytes = tiles * d * out_bytes;
+  s.q = 0;
+  s.k = s.q + round256(s.q_bytes);
+  s.v = s.k + round256(s.q_bytes);
+  s.alpha = s.v + round256(s.v_bytes);
+  s.beta = s.alpha + round256(s.alpha_bytes);
+  s.out = s.beta + round256(s.beta_bytes);
+  s.total = s.out + round256(s.out_bytes);
+  return s;
+}
+
 cudaError_t launch_decode(const KParams &p, cudaStream_t stream);
 cudaError_t launch_init(const KParams &p, cudaStream_t stream);
 cudaError_t launch_prefill(const KParams &p, cudaStream_t stream);

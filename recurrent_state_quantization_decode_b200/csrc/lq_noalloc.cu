@@ -11,16 +11,20 @@
 // The array below is a file-scope __device__ variable of
 // kNoallocStagingBytes (8 MiB): every GPU that loads the library holds it
 // until the process exits.  All calls share it, and it keeps the previous
-// call's contents; the output region is cleared on every call.  Calls that
-// overlap on the GPU (on different streams, or from different threads) race
-// on the array, so the caller must order them.
+// call's contents.  The step writes every output row it copies back (active
+// rows from the kernel; with an active mask, inactive rows are first filled
+// from the caller's own output buffer), so no stale bytes reach the caller.
+// Calls that overlap on the GPU (on different streams, or from different
+// threads) race on the array, so the caller must order them.
 //
 // Host code cannot use the array's name as a device address: in host code it
 // names a host-side stand-in.  The first call on each device therefore looks
 // the real address up with cudaGetSymbolAddress, with that device current, and
-// caches it; that first call should come before any stream capture.  Device
-// code in this file could name the array directly; only host code needs the
-// looked-up address.
+// caches it; that first call should come before any stream capture.  The
+// cached address belongs to the device's primary context: after
+// cudaDeviceReset the library must be reloaded before this entry point is
+// called again on that device.  Device code in this file could name the array
+// directly; only host code needs the looked-up address.
 
 #include <atomic>
 #include <cstdint>
@@ -28,7 +32,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/leapquant.h"
-#include "lq_internal.h"
+#include "lq_capi_internal.h"
 
 namespace {
 
@@ -39,17 +43,23 @@ static __device__ __align__(256) unsigned char g_noalloc_staging[kNoallocStaging
 
 std::atomic<void *> g_staging_addr[kMaxDevices];
 
-size_t round256(size_t x) { return (x + 255) / 256 * 256; }
-
 // Device address of the staging array on the current device (looked up once
-// per device).  Returns null if the lookup fails.
+// per device).  Returns null if the lookup fails; a failed lookup leaves no
+// sticky error behind for the next runtime call.
 void *staging_address() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
   void *p = g_staging_addr[dev].load(std::memory_order_acquire);
   if (p != nullptr) return p;
   void *addr = nullptr;
-  if (cudaGetSymbolAddress(&addr, g_noalloc_staging) != cudaSuccess) return nullptr;
+  if (cudaGetSymbolAddress(&addr, g_noalloc_staging) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
   g_staging_addr[dev].store(addr, std::memory_order_release);
   return addr;
 }
@@ -62,25 +72,14 @@ extern "C" lq_status lq_decode_step_host_noalloc(const lq_config *cfg, const voi
                                                  const float *beta_host, const lq_state *st,
                                                  void *out_host, const int32_t *active,
                                                  void *stream) {
-  lq_layout layout;
-  lq_status s = lq_state_layout(cfg, &layout);
+  // every argument is checked before the array is looked up or touched
+  lq_status s = lq::check_host_step(cfg, q_host, k_host, v_host, alpha_host, beta_host, st,
+                                    out_host, active);
   if (s != LQ_OK) return s;
-  if (layout.host_staging_bytes > kNoallocStagingBytes) return LQ_ERR_TOO_LARGE;
+  if (lq::host_staging_bytes(cfg) > kNoallocStagingBytes) return LQ_ERR_TOO_LARGE;
   if (cfg->batch == 0) return LQ_OK;
   void *staging = staging_address();
   if (staging == nullptr) return LQ_ERR_CUDA;
-  // The kernel writes outputs only for active sequences: clear the output
-  // region so inactive ones read back as zeros, not as an earlier call's data.
-  const size_t in_bytes = cfg->in_dtype == LQ_DTYPE_BF16 ? 2 : 4;
-  const size_t out_bytes = cfg->out_dtype == LQ_DTYPE_BF16 ? 2 : 4;
-  const size_t B = cfg->batch, Hk = cfg->num_k_heads, Hv = cfg->num_v_heads, d = cfg->d;
-  const size_t tiles = B * Hv, ga = cfg->gate == LQ_GATE_DIAG ? d : 1;
-  const size_t out_off = 2 * round256(B * Hk * d * in_bytes) + round256(tiles * d * in_bytes) +
-                         round256(tiles * ga * 4) + round256(tiles * 4);
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(static_cast<unsigned char *>(staging) + out_off, 0,
-                      tiles * d * out_bytes, cs) != cudaSuccess)
-    return LQ_ERR_CUDA;
   return lq_decode_step_host(cfg, q_host, k_host, v_host, alpha_host, beta_host, st, out_host,
                              staging, active, stream);
 }

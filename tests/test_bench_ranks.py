@@ -163,14 +163,20 @@ def test_algorithmic_bytes_and_profiled_traffic(tmp_path, monkeypatch):
     src = tmp_path / "kernel.cu"
     src.write_text("// kernel v1\n")
     monkeypatch.setattr(bench, "KERNEL_SOURCES", [str(src)])
-    summary = tmp_path / "summary.md"
-    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(summary))
+    summary = tmp_path / "decode_kernel_qwen35_9b_gdn.md"
+    monkeypatch.setattr(bench, "PROFILE_DIR", str(tmp_path))
+    assert bench.profile_summary_path("qwen35_9b_gdn") == str(summary)
     assert bench.profiled_traffic(10) is None                   # no summary
     summary.write_text(f"kernel_source_sha: {bench.kernel_source_sha()}\n"
                        "dram_bytes_per_tile_step: 24911\n")
     assert bench.profiled_traffic(2048) == 24911 * 2048
+    assert bench.profiled_traffic(4096, "kimi_linear_kda") is None   # another workload's file
     src.write_text("// kernel v2\n")                            # kernel changed since
     assert bench.profiled_traffic(2048) is None
+    # the roofline names the kernel instance of each workload
+    assert bench.kernel_label(bench.WORKLOADS["kimi_linear_kda"]).startswith(
+        "decode_kernel<128,bf16,KDA>")
+    assert bench.kernel_label(w).startswith("decode_kernel<128,bf16,GDN>")
 
 
 def test_working_set_and_l2_statement():

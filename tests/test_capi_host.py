@@ -151,6 +151,22 @@ def test_newer_entry_points_reject_bad_arguments_before_launch(B):
                 good + 8, stream=0) == B.LQ_ERR_MISALIGNED
     assert _err(B, B.lq_decode_step_host, cfg, good, good, good, good, good, st, good, good,
                 active=good + 1, stream=0) == B.LQ_ERR_MISALIGNED
+    # the no-alloc host step checks every argument before it looks up or
+    # touches its array: without a GPU these come back as argument errors,
+    # not as a CUDA error from the lookup
+    assert _err(B, B.lq_decode_step_host_noalloc, cfg, None, good, good, good, good, st,
+                good, stream=0) == B.LQ_ERR_INVALID_ARG
+    assert _err(B, B.lq_decode_step_host_noalloc, cfg, good, good, good, good, good, st,
+                good, active=good + 1, stream=0) == B.LQ_ERR_MISALIGNED
+    assert _err(B, B.lq_decode_step_host_noalloc, cfg, good + 4, good, good, good, good, st,
+                good, stream=0) == B.LQ_ERR_MISALIGNED
+    assert _err(B, B.lq_decode_step_host_noalloc, bad_cfg := B.make_config(2, 2, 4, 96), good,
+                good, good, good, good, st, good, stream=0) == B.LQ_ERR_UNSUPPORTED
+    big = B.make_config(4096, 32, 32, 128)        # staging above the fixed array
+    assert B.lq_state_layout(big).host_staging_bytes > B.LQ_NOALLOC_STAGING_MAX_BYTES
+    assert _err(B, B.lq_decode_step_host_noalloc, big, good, good, good, good, good, st, good,
+                stream=0) == B.LQ_ERR_TOO_LARGE
+    del bad_cfg
     # timeout hook: a zero poll limit or an empty batch is refused
     assert _err(B, B.lq_test_decode_step_timeout, cfg, good, good, good, good, good, st, good,
                 0, stream=0) == B.LQ_ERR_INVALID_ARG

@@ -95,6 +95,9 @@ CASES = {
                                        n_comp=8, smooth=1.0), 20),
     "naive_w1_k0": (wl.Workload("n", 1, 1, 2, 32, wl.GATE_SCALAR, False, 12, window=1,
                                 n_comp=0, smooth=0.0), 12),
+    "gdn_d128_f32": (wl.Workload("gf", 2, 2, 4, 128, wl.GATE_SCALAR, False, 36), 36),
+    "kda_d128_f32": (wl.Workload("kf", 2, 2, 2, 128, wl.GATE_DIAG, False, 36,
+                                 v_outlier_channels=4), 36),
 }
 
 
@@ -211,12 +214,28 @@ def test_fp32_path_vs_exact(case):
 # ragged batches: active masks and partial-window flushes
 # --------------------------------------------------------------------------
 
-def test_active_mask_and_flush():
-    """Ragged batch: random active masks and partial-window flushes.  Each
-    tile is teacher-forced at its own folds: whenever a tile's window closes
-    (boundary or flush), its record is compared and the oracle's is written
-    into the GPU state."""
-    w = wl.Workload("r", 5, 2, 4, 64, wl.GATE_DIAG, True, 48)
+RAGGED_CASES = {
+    # the general path: KDA, bf16 inputs, d = 64
+    "kda_d64_bf16": wl.Workload("r", 5, 2, 4, 64, wl.GATE_DIAG, True, 48),
+    # the path the bench times for GDN: bf16 inputs, d = 128, grouped heads
+    # (Hk = 16, Hv = 32), so tiles of one CTA sit in different window phases
+    "gdn_gva_d128_bf16": wl.Workload("rg", 5, 16, 32, 128, wl.GATE_SCALAR, True, 48),
+    # GDN with fp32 inputs at d = 128 (the general path at full width)
+    "gdn_d128_f32": wl.Workload("rf", 6, 4, 8, 128, wl.GATE_SCALAR, False, 48),
+    # KDA with bf16 inputs at d = 128 (the Kimi-Linear-like shape, fewer tiles)
+    "kda_d128_bf16": wl.Workload("rk", 5, 8, 8, 128, wl.GATE_DIAG, True, 48,
+                                 v_outlier_channels=4),
+}
+
+
+@pytest.mark.parametrize("case", sorted(RAGGED_CASES))
+def test_active_mask_and_flush(case):
+    """Ragged batch: random active masks and partial-window flushes, so that
+    the tiles of one launch (and of one CTA) sit in different window phases.
+    Each tile is teacher-forced at its own folds: whenever a tile's window
+    closes (boundary or flush), its record is compared and the oracle's is
+    written into the GPU state."""
+    w = RAGGED_CASES[case]
     T = 48
     rng = np.random.default_rng(7)
     S0, _, _ = wl.initial_states(rng, w.tiles, w.d, w.d)
@@ -225,7 +244,7 @@ def test_active_mask_and_flush():
     flush = rng.random((T, w.batch)) < 0.1
     cfg = B.config_for(w)
     ds, tiles = _init_both(w, cfg, S0)
-    dev = P.DeviceInputs(ti, True)
+    dev = P.DeviceInputs(ti, w.io_bf16)
     out = torch.empty((w.batch, w.num_v_heads, w.d), dtype=torch.float32, device="cuda")
     rv = ds.record_view()
     folds = 0
