@@ -135,6 +135,9 @@ struct SL {
 // leaves room for three ring slots at two CTAs per SM.
 template <int D, bool BF16, bool KDA>
 struct DecodeTraits {
+  // plain tokens (no fold) of d = 128 tiles with bf16 inputs run on the quad
+  // path: four warps per tile, two tiles at once per CTA
+  static constexpr bool kQuad = BF16 && D == 128;
   static constexpr bool kFast = BF16 && !KDA;
   static constexpr bool kKtOverCodes = kFast && kMaxWindow * FG<D>::PADW * 4 <= D * D;
   static constexpr int kStages = kFast ? 3 : 2;
@@ -192,17 +195,44 @@ struct Tok {
   float xscale[2][4];  // digit scales of x_q, x_k (per int8 k-chunk on the GDN-bf16 path)
 };
 
-template <int D, bool KT, int NT = 1>
-struct Scratch : KtArea<D, KT> {
+// Per-token values of the quad path, written by the quad's four warps before
+// its barrier and read by them after it.  Each quad keeps two, so that a warp
+// may start the next tile's channel work while the others finish the rows.
+template <int D>
+struct QTok {
+  alignas(16) int8_t dig[8][FG<D>::DIGW];  // digits: rows 0-3 of x_q, 4-7 of x_k
+  float xscale[2][4];                       // digit scale of each k-chunk (x_q, x_k)
+  float cpart[kMaxComp][4][2];              // row-compensator dots: one partial per warp
+  float colv[kMaxComp][2];                  // column compensator j: Gamma_j q_j, Gamma_j k_j
+  float cc[kMaxWindow + 1];                 // GDN: c_s = rho_s k_s . k
+  float aa[kMaxWindow + 1];                 // GDN: a_s = rho_s k_s . q
+  float rho[kMaxWindow + 1];                // GDN: decay ratios
+  float cpk[4][2 * kMaxWindow];             // KDA: per warp, partial c_s (s) and a_s (16 + s)
+};
+
+template <int D, int NT, bool Q>
+union TokArea {
   Tok<D> tok[NT];
+};
+template <int D, int NT>
+union TokArea<D, NT, true> {
+  Tok<D> tok[NT];     // the whole-CTA path
+  QTok<D> qt[2][2];   // the quad path: [quad][buffer]
+};
+
+template <int D, bool KT, int NT = 1, bool Q = false>
+struct Scratch : KtArea<D, KT> {
+  TokArea<D, NT, Q> u;
   alignas(16) float invm[FG<D>::PADW];             // 1 / m (new smoothing factors)
   alignas(16) float line[D];                       // the compensator line being extracted
   alignas(16) double rowE[D];
   unsigned long long pkey[kWarps];   // per-warp best selection key of the line energies
   int pid[kWarps];
   int abort;
-  int done[3];  // warps finished with each ring slot (GDN-bf16 path)
+  int done[3];       // warps finished with each ring slot (GDN-bf16 and quad paths)
+  int slot_last[3];  // list index of the last tile whose copies went into each slot
   int warp_cnt[kWarps];
+  int warp_cnt2[kWarps];
   int tl_tile[kMaxTilesPerCta];
   int tl_n[kMaxTilesPerCta];      // window phase; -1: skip (corrupt phase)
   int tl_coord[kMaxTilesPerCta];  // b << 12 | hk << 1 | (this value head writes the key)
@@ -1096,6 +1126,300 @@ __device__ __forceinline__ void channel_chunk_fast(const KParams &p, TK &x,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Quad path: plain tokens of d = 128 tiles with bf16 inputs
+// ---------------------------------------------------------------------------
+//
+// Four warps (a quad) take one tile: warp w of the quad does the per-channel
+// work of int8 k-chunk w (32 key channels) and then finishes the 32 state rows
+// 32w .. 32w + 31 (two m16 row blocks).  One named barrier per tile separates
+// the two phases; the per-token values go through a double-buffered QTok.  A
+// CTA runs two quads on two tiles at once, so the per-tile fixed costs (waits,
+// digit scales, combines, reductions) are spread over four warps instead of
+// eight, and no CTA-wide barrier is taken on a plain token.
+
+// Sums 32 per-lane values over the warp: afterwards lane l holds the total of
+// value l (31 shuffles).
+__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int step = 16, half = 16; step >= 1; step >>= 1, half >>= 1) {
+    const bool upper = (lane & step) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(kFull, send, step);
+    }
+  }
+  return v[0];
+}
+
+// Named barrier of one quad (128 threads, barrier id 1 + quad) that also
+// returns whether `pred` held in any of its threads.
+template <int ID>
+__device__ __forceinline__ bool bar_any_128(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "n"(ID)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool quad_bar_any(int quad, bool pred) {
+  return quad == 0 ? bar_any_128<1>(pred) : bar_any_128<2>(pred);
+}
+
+// Phase 1 of a quad tile, warp w (0..3) of the quad: k-chunk w's channels
+// 64(w/2) + 16(l/8) + 8(w%2) + l%8 for lane l.  Computes the window gate
+// Gamma (GDN: the scalar product of the gates; KDA: per channel, together with
+// this chunk's share of the buffer coefficients c_s = sum_j k_sj rho_sj k_j,
+// a_s = sum_j k_sj rho_sj q_j, rho_sj = prod_{s < s' <= n} alpha_s'j, and a_n =
+// k . q), x = m o Gamma o {q, k} and its digits under the chunk's own scale,
+// the row-compensator dots and the column-compensator values; warp 0 gets the
+// GDN coefficients from the bf16 tensor path.  Appends k_t (the key head's
+// first value head) and the gate when `ok` (the slot's copies arrived).
+template <int D, bool KDA>
+__device__ __forceinline__ void quad_channel(const KParams &p, QTok<D> &x, const uint8_t *slot,
+                                             int tile, int n, int coord, float alpha0, int w,
+                                             bool ok) {
+  using L = SL<D, true, KDA>;
+  const L lay(p.L.bytes);
+  const int lane = threadIdx.x & 31;
+  const int j = 64 * (w >> 1) + 16 * (lane >> 3) + 8 * (w & 1) + (lane & 7);
+  const float *rm = reinterpret_cast<const float *>(slot + p.L.off_m);
+  const float *rcv = reinterpret_cast<const float *>(slot + p.L.off_cv);
+  const int *rcid = reinterpret_cast<const int *>(slot + p.L.off_cid);
+  const __nv_bfloat16 *sbk = reinterpret_cast<const __nv_bfloat16 *>(slot + lay.bk);
+  const float *sbg = reinterpret_cast<const float *>(slot + lay.bg);
+  const __nv_bfloat16 *sq = reinterpret_cast<const __nv_bfloat16 *>(slot + lay.q);
+  const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(slot + lay.k);
+  const float q = __bfloat162float(sq[j]), k = __bfloat162float(sk[j]);
+  float G;
+  if constexpr (KDA) {
+    const float *sa = reinterpret_cast<const float *>(slot + lay.a);
+    // v[s]: this lane's share of c_s; v[16 + s]: of a_s (a_n = k . q)
+    float v[32];
+    float rho = sa[j];
+#pragma unroll
+    for (int s2 = kMaxWindow - 1; s2 >= 0; --s2) {
+      if (s2 < n) {
+        const float kr = __bfloat162float(sbk[s2 * D + j]) * rho;
+        v[s2] = kr * k;
+        v[16 + s2] = kr * q;
+        rho *= sbg[s2 * D + j];
+      } else {
+        v[s2] = 0.0f;
+        v[16 + s2] = (s2 == n) ? k * q : 0.0f;
+      }
+    }
+    G = rho;
+    x.cpk[w][lane] = warp_transpose_sum32(v, lane);
+  } else {
+    G = gate_product(sbg, alpha0, n);
+    if (w == 0)
+      coef_mma<D>(x, sbk, sk, sq, sbg, alpha0, n);
+  }
+  const float mj = rm[j];
+  const float gq = G * q, gk = G * k;
+  const float xq = mj * gq, xk = mj * gk;
+  const float mq = warp_max_abs(xq), mk = warp_max_abs(xk);
+  float upq = 0.0f, dnq = 0.0f, upk = 0.0f, dnk = 0.0f;
+  if (mq > 0.0f) digit_scales(mq, upq, dnq);
+  if (mk > 0.0f) digit_scales(mk, upk, dnk);
+  uint32_t dq[4] = {0u, 0u, 0u, 0u}, dk[4] = {0u, 0u, 0u, 0u};
+  digits4(xq * upq, dq, 0);
+  digits4(xk * upk, dk, 0);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    x.dig[r][j] = static_cast<int8_t>(dq[r]);
+    x.dig[4 + r][j] = static_cast<int8_t>(dk[r]);
+  }
+  if (lane == 0) {
+    x.xscale[0][w] = dnq;
+    x.xscale[1][w] = dnk;
+  }
+  // row-compensator lines: this chunk's share of their dots with Gamma o q and
+  // Gamma o k, four lines per transposed reduction; column lines: the owner
+  // lane of the column records Gamma_j q_j and Gamma_j k_j
+  for (int c0 = 0; c0 < p.K; c0 += 4) {
+    float vv[8];
+#pragma unroll
+    for (int i2 = 0; i2 < 4; ++i2) {
+      const int c = c0 + i2;
+      const float cvj = (c < p.K && rcid[c] < D) ? rcv[c * D + j] : 0.0f;
+      vv[2 * i2] = cvj * gq;
+      vv[2 * i2 + 1] = cvj * gk;
+    }
+    const float tot = warp_sum8(vv, lane);
+    const int vi = (lane >> 2) & 7, c = c0 + (vi >> 1);
+    if ((lane & 3) == 0 && c < p.K) x.cpart[c][w][vi & 1] = tot;
+  }
+  for (int c = 0; c < p.K; ++c) {
+    if (rcid[c] == D + j) {
+      x.colv[c][0] = gq;
+      x.colv[c][1] = gk;
+    }
+  }
+  if (ok) {
+    const int b = coord >> 12, hk = (coord >> 1) & 2047;
+    if ((coord & 1) != 0)
+      reinterpret_cast<__nv_bfloat16 *>(p.buf_k)[((static_cast<size_t>(b) * p.Hk + hk) * p.W + n) *
+                                                     D + j] = sk[j];
+    if constexpr (KDA) {
+      const float *sa = reinterpret_cast<const float *>(slot + lay.a);
+      p.buf_g[(static_cast<size_t>(tile) * p.W + n) * D + j] = sa[j];
+    } else {
+      if (w == 0 && lane == 0) p.buf_g[static_cast<size_t>(tile) * kGdnGateStride + n] = alpha0;
+    }
+  }
+}
+
+// Phase 2 of a quad tile, warp w: rows 32w .. 32w + 31 as two m16 row blocks.
+// y_q, y_k on the int8 tensor path with the four chunk scales, then the
+// buffer sums (lane t of a row takes slots t, t + 4, ...), the compensator
+// lines, d_t = beta (v - y_k - sum c_s d_s), o_t = y_q + sum a_s d_s + a_n d_t,
+// the output and the append of d_t.  A0 holds the first row block's codes.
+template <int D, bool KDA>
+__device__ __forceinline__ void quad_rows(const KParams &p, const QTok<D> &x, const uint8_t *slot,
+                                          int tile, int n, float beta, int w,
+                                          const uint4 (&A0)[2][2]) {
+  using L = SL<D, true, KDA>;
+  const L lay(p.L.bytes);
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const float *rsig = reinterpret_cast<const float *>(slot + p.L.off_sig);
+  const float *rcv = reinterpret_cast<const float *>(slot + p.L.off_cv);
+  const int *rcid = reinterpret_cast<const int *>(slot + p.L.off_cid);
+  const float *sbd = reinterpret_cast<const float *>(slot + lay.bd);
+  const __nv_bfloat16 *sv = reinterpret_cast<const __nv_bfloat16 *>(slot + lay.v);
+  // the coefficients of this lane's buffer slots s = t + 4u
+  float cs[4], as[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int s2 = t + 4 * u;
+    cs[u] = 0.0f;
+    as[u] = 0.0f;
+    if (s2 < n) {
+      if constexpr (KDA) {
+        cs[u] = (x.cpk[0][s2] + x.cpk[1][s2]) + (x.cpk[2][s2] + x.cpk[3][s2]);
+        as[u] = (x.cpk[0][16 + s2] + x.cpk[1][16 + s2]) + (x.cpk[2][16 + s2] + x.cpk[3][16 + s2]);
+      } else {
+        cs[u] = x.cc[s2];
+        as[u] = x.aa[s2];
+      }
+    }
+  }
+  float ann;
+  if constexpr (KDA)
+    ann = (x.cpk[0][16 + n] + x.cpk[1][16 + n]) + (x.cpk[2][16 + n] + x.cpk[3][16 + n]);
+  else
+    ann = x.aa[n];
+  uint4 Bw[2];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh)
+    Bw[hh] = *reinterpret_cast<const uint4 *>(&x.dig[g][frag_col(hh, t, 0)]);
+  const float pair = (t & 1) ? 1.0f / (128.0f * 16384.0f) : 1.0f / 128.0f;
+  float sc[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) sc[c] = x.xscale[t >> 1][c] * pair;
+  const int base_lane = lane & ~3;
+#pragma unroll
+  for (int rb2 = 0; rb2 < 2; ++rb2) {
+    const int r0 = 32 * w + 16 * rb2 + g, r1 = r0 + 8;
+    uint4 A[2][2];
+    if (rb2 == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        A[0][h] = A0[0][h];
+        A[1][h] = A0[1][h];
+      }
+    } else {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        A[0][h] = *reinterpret_cast<const uint4 *>(slot + r0 * D + frag_col(h, t, 0));
+        A[1][h] = *reinterpret_cast<const uint4 *>(slot + r1 * D + frag_col(h, t, 0));
+      }
+    }
+    int acc[4][4];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[2 * hh][e] = acc[2 * hh + 1][e] = 0;
+      mma_s8(acc[2 * hh], A[0][hh].x, A[1][hh].x, A[0][hh].y, A[1][hh].y, Bw[hh].x, Bw[hh].y);
+      mma_s8(acc[2 * hh + 1], A[0][hh].z, A[1][hh].z, A[0][hh].w, A[1][hh].w, Bw[hh].z,
+             Bw[hh].w);
+    }
+    float p0 = 0.0f, p1 = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      p0 = fmaf(sc[c], static_cast<float>(acc[c][0] * 128 + acc[c][1]), p0);
+      p1 = fmaf(sc[c], static_cast<float>(acc[c][2] * 128 + acc[c][3]), p1);
+    }
+    p0 += __shfl_xor_sync(kFull, p0, 1);
+    p1 += __shfl_xor_sync(kFull, p1, 1);
+    const float yq0 = __shfl_sync(kFull, p0, base_lane) * rsig[r0];
+    const float yq1 = __shfl_sync(kFull, p1, base_lane) * rsig[r1];
+    const float yk0 = __shfl_sync(kFull, p0, base_lane | 2) * rsig[r0];
+    const float yk1 = __shfl_sync(kFull, p1, base_lane | 2) * rsig[r1];
+    float xc0 = 0.0f, xa0 = 0.0f, xc1 = 0.0f, xa1 = 0.0f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int s2 = t + 4 * u;
+      if (s2 < n) {
+        const float d0 = sbd[s2 * D + r0], d1 = sbd[s2 * D + r1];
+        xc0 = fmaf(cs[u], d0, xc0);
+        xa0 = fmaf(as[u], d0, xa0);
+        xc1 = fmaf(cs[u], d1, xc1);
+        xa1 = fmaf(as[u], d1, xa1);
+      }
+    }
+    for (int c = t; c < p.K; c += 4) {
+      const int id = rcid[c];
+      if (id < D) {
+        if (id == r0 || id == r1) {
+          const float dq = (x.cpart[c][0][0] + x.cpart[c][1][0]) +
+                           (x.cpart[c][2][0] + x.cpart[c][3][0]);
+          const float dk = (x.cpart[c][0][1] + x.cpart[c][1][1]) +
+                           (x.cpart[c][2][1] + x.cpart[c][3][1]);
+          if (id == r0) {
+            xa0 += dq;
+            xc0 += dk;
+          } else {
+            xa1 += dq;
+            xc1 += dk;
+          }
+        }
+      } else {
+        const float gq = x.colv[c][0], gk = x.colv[c][1];
+        const float c0 = rcv[c * D + r0], c1 = rcv[c * D + r1];
+        xa0 = fmaf(c0, gq, xa0);
+        xc0 = fmaf(c0, gk, xc0);
+        xa1 = fmaf(c1, gq, xa1);
+        xc1 = fmaf(c1, gk, xc1);
+      }
+    }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      xc0 += __shfl_xor_sync(kFull, xc0, o);
+      xa0 += __shfl_xor_sync(kFull, xa0, o);
+      xc1 += __shfl_xor_sync(kFull, xc1, o);
+      xa1 += __shfl_xor_sync(kFull, xa1, o);
+    }
+    if (t < 2) {
+      const int row = t ? r1 : r0;
+      const float yq = t ? yq1 : yq0, yk = t ? yk1 : yk0;
+      const float xc = t ? xc1 : xc0, xa = t ? xa1 : xa0;
+      const float dt = beta * (__bfloat162float(sv[row]) - yk - xc);
+      const float o = fmaf(ann, dt, yq + xa);
+      st_out(p.out, static_cast<size_t>(tile) * D + row, o, p.out_bf16);
+      p.buf_d[(static_cast<size_t>(tile) * p.W + n) * D + row] = dt;
+    }
+  }
+}
+
 // One token for one staged tile: outputs, buffer append, and on the W-th token
 // the fold and requantization.
 // GDN with bf16 inputs (one CTA barrier; returns false if the CTA aborts):
@@ -1452,30 +1776,48 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
   return true;
 }
 
+// Bounded wait until the slot's last issued list entry is at least `e`;
+// false after `limit` polls.
+__device__ __forceinline__ bool wait_issued(const int *slot_last, int e, uint32_t limit) {
+  for (uint32_t it = 0; it < limit; ++it)
+    if (*reinterpret_cast<const volatile int *>(slot_last) >= e) return true;
+  return false;
+}
+
+// L2 prefetch of `bytes` at `src` (16-byte aligned, a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 template <int D, bool BF16, bool KDA>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
   using L = SL<D, BF16, KDA>;
   using TR = DecodeTraits<D, BF16, KDA>;
   constexpr int kStages = TR::kStages;
-  using SC = Scratch<D, !TR::kKtOverCodes, TR::kTok>;
+  constexpr bool kQuad = TR::kQuad;
+  using SC = Scratch<D, !TR::kKtOverCodes, TR::kTok, kQuad>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int slot_bytes = L(p.L.bytes).bytes;
   SC &s = *reinterpret_cast<SC *>(smem + kStages * slot_bytes);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tiles = p.B * p.Hv;
 
-  // This CTA's tiles are blockIdx.x + i * gridDim.x.  Without a mask every
-  // tile keeps its position in the list, so the first slots' record copies go
-  // out before the phases are known; with a mask the list is compacted to the
-  // active sequences first.
+  // This CTA's tiles are blockIdx.x + i * gridDim.x.  The list is built in
+  // that order, compacted to the active sequences when there is a mask; on
+  // the quad path the plain tokens (0 <= n < W - 1) come first and the rest
+  // (boundary tokens, skipped tiles) after them.  Without a mask and without
+  // the quad path every tile keeps its position, so the first slots' record
+  // copies go out before the phases are known; the quad path prefetches
+  // those records into L2 instead.
   const int mine = (tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
-  const bool speculate = p.mask == nullptr;
+  const bool speculate = !kQuad && p.mask == nullptr;
   if (tid == 0) {
     s.abort = 0;
     for (int st = 0; st < kStages; ++st) {
       mbar_init(&s.bar[st], 1);
       s.done[st] = 0;
+      s.slot_last[st] = -1;
     }
     fence_mbar_init();
   }
@@ -1486,11 +1828,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
-    if (speculate)
-      for (int st = 0; st < kStages && st < mine; ++st)
+    for (int st = 0; st < kStages && st < mine; ++st) {
+      const int tl = blockIdx.x + st * gridDim.x;
+      if (speculate) {
         if (!(p.withhold && blockIdx.x == 0 && st == 0))
-          issue_record<D, BF16, KDA>(p, smem + st * slot_bytes, &s.bar[st],
-                                     blockIdx.x + st * gridDim.x);
+          issue_record<D, BF16, KDA>(p, smem + st * slot_bytes, &s.bar[st], tl);
+      } else if (kQuad) {
+        prefetch_l2(p.records + static_cast<size_t>(tl) * p.L.bytes,
+                    static_cast<uint32_t>(p.L.bytes));
+      }
+    }
   }
   int keep = 0, tile = 0, n = -1, coord = 0;
   float a0 = 0.0f, b0 = 0.0f;
@@ -1498,7 +1845,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
     tile = blockIdx.x + tid * gridDim.x;
     const int b = tile / p.Hv, h = tile - b * p.Hv, group = p.Hv / p.Hk;
     coord = (b << 12) | ((h / group) << 1) | ((h % group == 0) ? 1 : 0);
-    if (speculate || p.mask[b] != 0) {
+    if (speculate || p.mask == nullptr || p.mask[b] != 0) {
       keep = 1;
       n = p.buf_n[tile];
       if (n >= 0 && n < p.W) {
@@ -1510,17 +1857,26 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
       }
     }
   }
-  const unsigned ball = __ballot_sync(kFull, keep);
-  if (lane == 0) s.warp_cnt[warp] = __popc(ball);
+  const bool plain = kQuad && keep && n >= 0 && n < p.W - 1;
+  const unsigned ball_p = __ballot_sync(kFull, plain);
+  const unsigned ball_o = __ballot_sync(kFull, keep && !plain);
+  if (lane == 0) {
+    s.warp_cnt[warp] = __popc(ball_p);
+    s.warp_cnt2[warp] = __popc(ball_o);
+  }
   __syncthreads();
-  int base = 0, count = 0;
+  int base_p = 0, base_o = 0, P = 0, count = 0;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
-    base += (w < warp) ? s.warp_cnt[w] : 0;
-    count += s.warp_cnt[w];
+    base_p += (w < warp) ? s.warp_cnt[w] : 0;
+    base_o += (w < warp) ? s.warp_cnt2[w] : 0;
+    P += s.warp_cnt[w];
+    count += s.warp_cnt2[w];
   }
+  count += P;
   if (keep) {
-    const int pos = base + __popc(ball & ((1u << lane) - 1u));
+    const unsigned below = (1u << lane) - 1u;
+    const int pos = plain ? base_p + __popc(ball_p & below) : P + base_o + __popc(ball_o & below);
     s.tl_tile[pos] = tile;
     s.tl_n[pos] = n;
     s.tl_coord[pos] = coord;
@@ -1529,33 +1885,97 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
   }
   __syncthreads();
 
+  // Copies of list entry `nx` into slot `st` (one thread).
+  auto issue = [&](int st, int nx) {
+    uint8_t *slot = smem + st * slot_bytes;
+    issue_record<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[nx]);
+    issue_rest<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[nx], s.tl_n[nx], s.tl_coord[nx]);
+    s.slot_last[st] = nx;
+  };
   if (tid == 0)
     for (int st = 0; st < kStages && st < count; ++st) {
-      uint8_t *slot = smem + st * slot_bytes;
       // testing: CTA 0 leaves its first slot without copies, so that the
       // bounded wait on it expires (nothing is in flight into that slot)
       if (p.withhold && blockIdx.x == 0 && st == 0) continue;
-      if (!speculate) issue_record<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[st]);
-      issue_rest<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[st], s.tl_n[st], s.tl_coord[st]);
+      if (speculate) {
+        uint8_t *slot = smem + st * slot_bytes;
+        issue_rest<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[st], s.tl_n[st],
+                                 s.tl_coord[st]);
+        s.slot_last[st] = st;
+      } else {
+        issue(st, st);
+      }
     }
-  // tiles whose copies have been issued (the same value in every thread)
-  int issued = count < kStages ? count : kStages;
+
+  bool aborted = false;
+  int i = 0;
+  if constexpr (kQuad) {
+    // Plain tokens, list entries 0 .. P-1: quad q takes entries q, q + 2, ...
+    // Entry i sits in slot i % kStages; the last warp of its quad to finish
+    // refills that slot with entry i + kStages.
+    const int quad = warp >> 2, w = warp & 3;
+    int li = 0;
+    bool qabort = false;
+    for (int e = quad; e < P; e += 2, ++li) {
+      const int st = e % kStages;
+      const uint32_t parity = static_cast<uint32_t>(e / kStages) & 1u;
+      // The two quads take alternate entries, so one may reach entry e while
+      // the entry before it in the same slot (e - kStages, the other quad's)
+      // is still unfinished and e not yet issued.  A parity wait alone could
+      // then pass on the earlier phase: first wait (bounded) until entry e's
+      // copies have been issued into the slot.
+      const bool ok = wait_issued(&s.slot_last[st], e, p.wait_limit) &&
+                      mbar_wait_bounded(&s.bar[st], parity, p.wait_limit);
+      uint8_t *slot = smem + st * slot_bytes;
+      QTok<D> &x = s.u.qt[quad][li & 1];
+      const int tl = s.tl_tile[e], ne = s.tl_n[e];
+      // the first row block's codes, fetched before the barrier
+      uint4 A0[2][2];
+      {
+        const int r0 = 32 * w + (lane >> 2), t = lane & 3;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          A0[0][h] = *reinterpret_cast<const uint4 *>(slot + r0 * D + frag_col(h, t, 0));
+          A0[1][h] = *reinterpret_cast<const uint4 *>(slot + (r0 + 8) * D + frag_col(h, t, 0));
+        }
+      }
+      quad_channel<D, KDA>(p, x, slot, tl, ne, s.tl_coord[e], s.tl_a[e], w, ok);
+      // the quad's one barrier per tile; it also tells every warp whether any
+      // thread's wait expired, so that the quad leaves the loop together
+      if (quad_bar_any(quad, !ok)) {
+        qabort = true;
+        break;
+      }
+      quad_rows<D, KDA>(p, x, slot, tl, ne, s.tl_b[e], w, A0);
+      if (w == 0 && lane == 0) p.buf_n[tl] = ne + 1;
+      // This warp is done with the slot: order its generic-proxy accesses
+      // before the bulk copy that refills it.
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        if (atomicAdd(&s.done[st], 1) == 3) {
+          s.done[st] = 0;
+          __threadfence_block();
+          if (e + kStages < count) issue(st, e + kStages);
+        }
+      }
+      __syncwarp();
+    }
+    aborted = __syncthreads_or(qabort) != 0;
+    i = P;
+  }
+
+  // The whole CTA on the remaining entries (every entry without the quad path).
+  int issued = count < i + kStages ? count : i + kStages;
   auto refill = [&](int freed) {
     // slot freed % kStages takes the next tile in line
     if (freed >= 0 && issued < count) {
-      if (tid == 0) {
-        uint8_t *slot = smem + (freed % kStages) * slot_bytes;
-        const int nx = issued;
-        issue_record<D, BF16, KDA>(p, slot, &s.bar[freed % kStages], s.tl_tile[nx]);
-        issue_rest<D, BF16, KDA>(p, slot, &s.bar[freed % kStages], s.tl_tile[nx], s.tl_n[nx],
-                                 s.tl_coord[nx]);
-      }
+      if (tid == 0) issue(freed % kStages, issued);
       ++issued;
     }
   };
-
-  int i = 0;
-  for (; i < count; ++i) {
+  for (; i < count && !aborted; ++i) {
     const int st = i % kStages;
     const uint32_t parity = static_cast<uint32_t>(i / kStages) & 1u;
     if constexpr (TR::kTok == 2) {
@@ -1565,14 +1985,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
       if (!mbar_wait_bounded(&s.bar[st], parity, p.wait_limit)) s.abort = 1;
       bool ok;
       if (s.tl_n[i] >= 0) {
-        ok = process_tile<D, BF16, KDA>(p, s, s.tok[i & 1], smem + st * slot_bytes,
+        ok = process_tile<D, BF16, KDA>(p, s, s.u.tok[i & 1], smem + st * slot_bytes,
                                         s.tl_tile[i], s.tl_n[i], s.tl_coord[i], s.tl_a[i],
                                         s.tl_b[i], [] {});
       } else {
         __syncthreads();
         ok = !s.abort;
       }
-      if (!ok) break;
+      if (!ok) {
+        aborted = true;
+        break;
+      }
       // This warp is done with the slot.  Its generic-proxy accesses are
       // ordered before the bulk copy that refills it; the last warp to finish
       // issues that copy (tile i + kStages) at once.
@@ -1583,39 +2006,38 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
         if (atomicAdd(&s.done[st], 1) == kWarps - 1) {
           s.done[st] = 0;
           __threadfence_block();
-          const int nx = i + kStages;
-          if (nx < count) {
-            uint8_t *slot = smem + st * slot_bytes;
-            issue_record<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[nx]);
-            issue_rest<D, BF16, KDA>(p, slot, &s.bar[st], s.tl_tile[nx], s.tl_n[nx],
-                                     s.tl_coord[nx]);
-          }
+          if (i + kStages < count) issue(st, i + kStages);
         }
       }
       __syncwarp();
     } else {
       if (!mbar_wait_bounded(&s.bar[st], parity, p.wait_limit)) s.abort = 1;
       __syncthreads();
-      if (s.abort) break;
+      if (s.abort) {
+        aborted = true;
+        break;
+      }
       if (s.tl_n[i] >= 0)
-        process_tile<D, BF16, KDA>(p, s, s.tok[0], smem + st * slot_bytes, s.tl_tile[i],
+        process_tile<D, BF16, KDA>(p, s, s.u.tok[0], smem + st * slot_bytes, s.tl_tile[i],
                                    s.tl_n[i], s.tl_coord[i], s.tl_a[i], s.tl_b[i], [] {});
       fence_proxy_async();
       __syncthreads();
       refill(i);
     }
   }
-  if (i < count) {
+  if (aborted) {
     // A copy did not complete in time: flag it, then give the copies still in
-    // flight into this CTA's shared memory a bounded chance to land.  On the
-    // GDN-bf16 path every tile before i had all its warps finish, so its
-    // slot's refill (tile + kStages) has been issued.
-    if constexpr (TR::kTok == 2) issued = (i + kStages < count) ? i + kStages : count;
+    // flight into this CTA's shared memory (the last ones issued into each
+    // slot) a bounded chance to land before the CTA exits.
+    __syncthreads();
     if (tid == 0) {
       atomicOr(p.err, kErrTimeout);
-      for (int k = i; k < issued; ++k)
-        mbar_wait_bounded(&s.bar[k % kStages], static_cast<uint32_t>(k / kStages) & 1u,
-                          p.wait_limit);
+      for (int st = 0; st < kStages; ++st) {
+        const int last = s.slot_last[st];
+        if (last >= 0)
+          mbar_wait_bounded(&s.bar[st], static_cast<uint32_t>(last / kStages) & 1u,
+                            p.wait_limit);
+      }
     }
     __syncthreads();
   }
@@ -1660,7 +2082,7 @@ __global__ void __launch_bounds__(kThreads) fold_kernel(const KParams p) {
   uint8_t *slot = smem;
   const L lay(p.L.bytes);
   Scratch<D, true> &s = *reinterpret_cast<Scratch<D, true> *>(smem + lay.bytes);
-  Tok<D> &x = s.tok[0];
+  Tok<D> &x = s.u.tok[0];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int tile = blockIdx.x;
@@ -1775,7 +2197,7 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const KParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t *qscr = smem;  // D*D bytes of quantizer scratch
   Scratch<D, false> &s = *reinterpret_cast<Scratch<D, false> *>(smem + D * D);
-  Tok<D> &x = s.tok[0];
+  Tok<D> &x = s.u.tok[0];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int tile = blockIdx.x;
@@ -1950,7 +2372,7 @@ cudaError_t decode_t(const KParams &p, cudaStream_t st) {
   using L = SL<D, BF16, KDA>;
   using TR = DecodeTraits<D, BF16, KDA>;
   constexpr int NST = TR::kStages;
-  constexpr size_t scratch = sizeof(Scratch<D, !TR::kKtOverCodes, TR::kTok>);
+  constexpr size_t scratch = sizeof(Scratch<D, !TR::kKtOverCodes, TR::kTok, TR::kQuad>);
   const size_t smem = NST * L(p.L.bytes).bytes + scratch;
   const size_t smem_max = NST * L(record_layout(D, kMaxComp).bytes).bytes + scratch;
   LaunchInfo li;
