@@ -138,6 +138,10 @@ struct DecodeTraits {
   // plain tokens (no fold) of d = 128 tiles with bf16 inputs run on the quad
   // path: four warps per tile, two tiles at once per CTA
   static constexpr bool kQuad = BF16 && D == 128;
+  // with one ring slot per quad (KDA), the quad releases its slot at its
+  // barrier, after loading the row-phase operands into registers
+  static constexpr bool kEarlyRelease = kQuad && KDA;
+  static_assert(kEarlyRelease == (kQuad && KDA), "one ring slot per quad only on KDA");
   static constexpr bool kFast = BF16 && !KDA;
   static constexpr bool kKtOverCodes = kFast && kMaxWindow * FG<D>::PADW * 4 <= D * D;
   static constexpr int kStages = kFast ? 3 : 2;
@@ -365,11 +369,20 @@ __device__ __forceinline__ void mma_tf32(float2 &c01, float2 &c23, uint32_t a0, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Rounds a finite fp32 value to tf32 (10 explicit mantissa bits), to nearest
+// with ties away from zero: adding half of the last kept bit to the
+// magnitude's bit pattern carries into the kept bits exactly when the dropped
+// part is at least half of it, and the mask drops the rest.  Integer ALU work
+// only, in place of a conversion instruction.
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
+}
+
 // x = hi + lo with hi, lo tf32 (round to nearest); hi * hi' + hi * lo' + lo * hi'
-// then reproduces an fp32 product to about 2^-22 relative.
+// then reproduces an fp32 product to about 2^-22 relative.  x - hi is exact.
 __device__ __forceinline__ void tf32_split(float x, uint32_t &hi, uint32_t &lo) {
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(x - __uint_as_float(hi)));
+  hi = tf32_rna(x);
+  lo = tf32_rna(x - __uint_as_float(hi));
 }
 
 // Exact split of x into four radix-128 digits with the power-of-two scale
@@ -1278,15 +1291,23 @@ __device__ __forceinline__ void quad_channel(const KParams &p, QTok<D> &x, const
   }
 }
 
-// Phase 2 of a quad tile, warp w: rows 32w .. 32w + 31 as two m16 row blocks.
-// y_q, y_k on the int8 tensor path with the four chunk scales, then the
-// buffer sums (lane t of a row takes slots t, t + 4, ...), the compensator
-// lines, d_t = beta (v - y_k - sum c_s d_s), o_t = y_q + sum a_s d_s + a_n d_t,
-// the output and the append of d_t.  A0 holds the first row block's codes.
+// What phase 2 of a quad tile needs from the ring slot, held in registers so
+// that the slot can be refilled before the rows are computed.  Lane (g, t) of
+// warp w owns rows 32w + 16rb + g and + 8 (rb = 0, 1), the buffer slots
+// t, t + 4, ... of them, and the compensator lines t and t + 4.
+struct QRegs {
+  uint4 A[2][2][2];      // codes: [rb][row r0 / r1][64-column span]
+  float sig[2][2];       // sigma at the rows
+  float v[2];            // v at the row this lane finishes (t < 2), per rb
+  float d[4][2][2];      // d_s at the rows for s = t + 4u: [u][rb][r0 / r1]
+  int cid[2];            // ids of lines t and t + 4 (D2 + 1 past K)
+  float cval[2][2][2];   // those lines' values at the rows (column lines)
+};
+
+// Loads the QRegs of warp w for a tile with n buffered tokens from its slot.
 template <int D, bool KDA>
-__device__ __forceinline__ void quad_rows(const KParams &p, const QTok<D> &x, const uint8_t *slot,
-                                          int tile, int n, float beta, int w,
-                                          const uint4 (&A0)[2][2]) {
+__device__ __forceinline__ void quad_rows_load(const KParams &p, const uint8_t *slot, int n, int w,
+                                               QRegs &r) {
   using L = SL<D, true, KDA>;
   const L lay(p.L.bytes);
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -1295,6 +1316,107 @@ __device__ __forceinline__ void quad_rows(const KParams &p, const QTok<D> &x, co
   const int *rcid = reinterpret_cast<const int *>(slot + p.L.off_cid);
   const float *sbd = reinterpret_cast<const float *>(slot + lay.bd);
   const __nv_bfloat16 *sv = reinterpret_cast<const __nv_bfloat16 *>(slot + lay.v);
+#pragma unroll
+  for (int rb = 0; rb < 2; ++rb) {
+    const int r0 = 32 * w + 16 * rb + g, r1 = r0 + 8;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      r.A[rb][0][h] = *reinterpret_cast<const uint4 *>(slot + r0 * D + frag_col(h, t, 0));
+      r.A[rb][1][h] = *reinterpret_cast<const uint4 *>(slot + r1 * D + frag_col(h, t, 0));
+    }
+    r.sig[rb][0] = rsig[r0];
+    r.sig[rb][1] = rsig[r1];
+    r.v[rb] = __bfloat162float(sv[t ? r1 : r0]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int s2 = t + 4 * u;
+      r.d[u][rb][0] = s2 < n ? sbd[s2 * D + r0] : 0.0f;
+      r.d[u][rb][1] = s2 < n ? sbd[s2 * D + r1] : 0.0f;
+    }
+  }
+#pragma unroll
+  for (int li = 0; li < 2; ++li) {
+    const int c = t + 4 * li;
+    const int id = c < p.K ? rcid[c] : 2 * D + 1;
+    r.cid[li] = id;
+    const bool col = id >= D && id < 2 * D;
+#pragma unroll
+    for (int rb = 0; rb < 2; ++rb) {
+      const int r0 = 32 * w + 16 * rb + g;
+      r.cval[li][rb][0] = col ? rcv[c * D + r0] : 0.0f;
+      r.cval[li][rb][1] = col ? rcv[c * D + r0 + 8] : 0.0f;
+    }
+  }
+}
+
+// Row-phase operands as quad_rows reads them: from registers loaded before
+// the slot was released (RegRows), or from the slot when they are used
+// (SlotRows, for a ring whose other slots already overlap the copies with the
+// rows and where holding them all would cost registers).
+struct RegRows {
+  QRegs r;
+  __device__ __forceinline__ uint4 A(int rb, int rr, int h) const { return r.A[rb][rr][h]; }
+  __device__ __forceinline__ float sig(int rb, int rr) const { return r.sig[rb][rr]; }
+  __device__ __forceinline__ float v(int rb) const { return r.v[rb]; }
+  __device__ __forceinline__ float d(int u, int rb, int rr) const { return r.d[u][rb][rr]; }
+  __device__ __forceinline__ int cid(int li) const { return r.cid[li]; }
+  __device__ __forceinline__ float cval(int li, int rb, int rr) const { return r.cval[li][rb][rr]; }
+};
+
+template <int D, bool KDA>
+struct SlotRows {
+  const uint8_t *slot;
+  const float *rsig, *rcv, *sbd;
+  const int *rcid;
+  const __nv_bfloat16 *sv;
+  int n, K, row0, t;
+  __device__ __forceinline__ SlotRows(const KParams &p, const uint8_t *slot_, int n_, int w) {
+    using L = SL<D, true, KDA>;
+    const L lay(p.L.bytes);
+    const int lane = threadIdx.x & 31;
+    slot = slot_;
+    rsig = reinterpret_cast<const float *>(slot + p.L.off_sig);
+    rcv = reinterpret_cast<const float *>(slot + p.L.off_cv);
+    rcid = reinterpret_cast<const int *>(slot + p.L.off_cid);
+    sbd = reinterpret_cast<const float *>(slot + lay.bd);
+    sv = reinterpret_cast<const __nv_bfloat16 *>(slot + lay.v);
+    n = n_;
+    K = p.K;
+    row0 = 32 * w + (lane >> 2);
+    t = lane & 3;
+  }
+  __device__ __forceinline__ int row(int rb, int rr) const { return row0 + 16 * rb + 8 * rr; }
+  __device__ __forceinline__ uint4 A(int rb, int rr, int h) const {
+    return *reinterpret_cast<const uint4 *>(slot + row(rb, rr) * D + frag_col(h, t, 0));
+  }
+  __device__ __forceinline__ float sig(int rb, int rr) const { return rsig[row(rb, rr)]; }
+  __device__ __forceinline__ float v(int rb) const {
+    return __bfloat162float(sv[row(rb, t ? 1 : 0)]);
+  }
+  __device__ __forceinline__ float d(int u, int rb, int rr) const {
+    const int s2 = t + 4 * u;
+    return s2 < n ? sbd[s2 * D + row(rb, rr)] : 0.0f;
+  }
+  __device__ __forceinline__ int cid(int li) const {
+    const int c = t + 4 * li;
+    return c < K ? rcid[c] : 2 * D + 1;
+  }
+  __device__ __forceinline__ float cval(int li, int rb, int rr) const {
+    const int c = t + 4 * li, id = cid(li);
+    return (id >= D && id < 2 * D) ? rcv[c * D + row(rb, rr)] : 0.0f;
+  }
+};
+
+// Phase 2 of a quad tile, warp w: rows 32w .. 32w + 31 as two m16 row blocks,
+// from the QRegs and the quad's QTok only (the slot may already be refilled).
+// y_q, y_k on the int8 tensor path with the four chunk scales, then the
+// buffer sums (lane t of a row takes slots t, t + 4, ...), the compensator
+// lines (lane t takes lines t and t + 4), d_t = beta (v - y_k - sum c_s d_s),
+// o_t = y_q + sum a_s d_s + a_n d_t, the output and the append of d_t.
+template <int D, bool KDA, class Src>
+__device__ __forceinline__ void quad_rows(const KParams &p, const QTok<D> &x, const Src &r,
+                                          int tile, int n, float beta, int w) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   // the coefficients of this lane's buffer slots s = t + 4u
   float cs[4], as[4];
 #pragma unroll
@@ -1317,6 +1439,23 @@ __device__ __forceinline__ void quad_rows(const KParams &p, const QTok<D> &x, co
     ann = (x.cpk[0][16 + n] + x.cpk[1][16 + n]) + (x.cpk[2][16 + n] + x.cpk[3][16 + n]);
   else
     ann = x.aa[n];
+  // this lane's compensator lines: column lines scale their values at the rows
+  // by Gamma_j x_j; a row line adds its dots to the one row it is
+  float cq[2], ck[2], rq[2], rk[2];
+#pragma unroll
+  for (int li = 0; li < 2; ++li) {
+    const int c = t + 4 * li, id = r.cid(li);
+    cq[li] = ck[li] = rq[li] = rk[li] = 0.0f;
+    if (id < D) {
+      if ((id >> 5) == w) {
+        rq[li] = (x.cpart[c][0][0] + x.cpart[c][1][0]) + (x.cpart[c][2][0] + x.cpart[c][3][0]);
+        rk[li] = (x.cpart[c][0][1] + x.cpart[c][1][1]) + (x.cpart[c][2][1] + x.cpart[c][3][1]);
+      }
+    } else if (id < 2 * D) {
+      cq[li] = x.colv[c][0];
+      ck[li] = x.colv[c][1];
+    }
+  }
   uint4 Bw[2];
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh)
@@ -1327,30 +1466,16 @@ __device__ __forceinline__ void quad_rows(const KParams &p, const QTok<D> &x, co
   for (int c = 0; c < 4; ++c) sc[c] = x.xscale[t >> 1][c] * pair;
   const int base_lane = lane & ~3;
 #pragma unroll
-  for (int rb2 = 0; rb2 < 2; ++rb2) {
-    const int r0 = 32 * w + 16 * rb2 + g, r1 = r0 + 8;
-    uint4 A[2][2];
-    if (rb2 == 0) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        A[0][h] = A0[0][h];
-        A[1][h] = A0[1][h];
-      }
-    } else {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        A[0][h] = *reinterpret_cast<const uint4 *>(slot + r0 * D + frag_col(h, t, 0));
-        A[1][h] = *reinterpret_cast<const uint4 *>(slot + r1 * D + frag_col(h, t, 0));
-      }
-    }
+  for (int rb = 0; rb < 2; ++rb) {
+    const int r0 = 32 * w + 16 * rb + g, r1 = r0 + 8;
     int acc[4][4];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
+      const uint4 a0 = r.A(rb, 0, hh), a1 = r.A(rb, 1, hh);
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[2 * hh][e] = acc[2 * hh + 1][e] = 0;
-      mma_s8(acc[2 * hh], A[0][hh].x, A[1][hh].x, A[0][hh].y, A[1][hh].y, Bw[hh].x, Bw[hh].y);
-      mma_s8(acc[2 * hh + 1], A[0][hh].z, A[1][hh].z, A[0][hh].w, A[1][hh].w, Bw[hh].z,
-             Bw[hh].w);
+      mma_s8(acc[2 * hh], a0.x, a1.x, a0.y, a1.y, Bw[hh].x, Bw[hh].y);
+      mma_s8(acc[2 * hh + 1], a0.z, a1.z, a0.w, a1.w, Bw[hh].z, Bw[hh].w);
     }
     float p0 = 0.0f, p1 = 0.0f;
 #pragma unroll
@@ -1360,45 +1485,33 @@ __device__ __forceinline__ void quad_rows(const KParams &p, const QTok<D> &x, co
     }
     p0 += __shfl_xor_sync(kFull, p0, 1);
     p1 += __shfl_xor_sync(kFull, p1, 1);
-    const float yq0 = __shfl_sync(kFull, p0, base_lane) * rsig[r0];
-    const float yq1 = __shfl_sync(kFull, p1, base_lane) * rsig[r1];
-    const float yk0 = __shfl_sync(kFull, p0, base_lane | 2) * rsig[r0];
-    const float yk1 = __shfl_sync(kFull, p1, base_lane | 2) * rsig[r1];
+    const float yq0 = __shfl_sync(kFull, p0, base_lane) * r.sig(rb, 0);
+    const float yq1 = __shfl_sync(kFull, p1, base_lane) * r.sig(rb, 1);
+    const float yk0 = __shfl_sync(kFull, p0, base_lane | 2) * r.sig(rb, 0);
+    const float yk1 = __shfl_sync(kFull, p1, base_lane | 2) * r.sig(rb, 1);
     float xc0 = 0.0f, xa0 = 0.0f, xc1 = 0.0f, xa1 = 0.0f;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int s2 = t + 4 * u;
-      if (s2 < n) {
-        const float d0 = sbd[s2 * D + r0], d1 = sbd[s2 * D + r1];
-        xc0 = fmaf(cs[u], d0, xc0);
-        xa0 = fmaf(as[u], d0, xa0);
-        xc1 = fmaf(cs[u], d1, xc1);
-        xa1 = fmaf(as[u], d1, xa1);
-      }
+      const float d0 = r.d(u, rb, 0), d1 = r.d(u, rb, 1);
+      xc0 = fmaf(cs[u], d0, xc0);
+      xa0 = fmaf(as[u], d0, xa0);
+      xc1 = fmaf(cs[u], d1, xc1);
+      xa1 = fmaf(as[u], d1, xa1);
     }
-    for (int c = t; c < p.K; c += 4) {
-      const int id = rcid[c];
-      if (id < D) {
-        if (id == r0 || id == r1) {
-          const float dq = (x.cpart[c][0][0] + x.cpart[c][1][0]) +
-                           (x.cpart[c][2][0] + x.cpart[c][3][0]);
-          const float dk = (x.cpart[c][0][1] + x.cpart[c][1][1]) +
-                           (x.cpart[c][2][1] + x.cpart[c][3][1]);
-          if (id == r0) {
-            xa0 += dq;
-            xc0 += dk;
-          } else {
-            xa1 += dq;
-            xc1 += dk;
-          }
-        }
-      } else {
-        const float gq = x.colv[c][0], gk = x.colv[c][1];
-        const float c0 = rcv[c * D + r0], c1 = rcv[c * D + r1];
-        xa0 = fmaf(c0, gq, xa0);
-        xc0 = fmaf(c0, gk, xc0);
-        xa1 = fmaf(c1, gq, xa1);
-        xc1 = fmaf(c1, gk, xc1);
+#pragma unroll
+    for (int li = 0; li < 2; ++li) {
+      const float v0 = r.cval(li, rb, 0), v1 = r.cval(li, rb, 1);
+      xa0 = fmaf(v0, cq[li], xa0);
+      xc0 = fmaf(v0, ck[li], xc0);
+      xa1 = fmaf(v1, cq[li], xa1);
+      xc1 = fmaf(v1, ck[li], xc1);
+      const int id = r.cid(li);
+      if (id == r0) {
+        xa0 += rq[li];
+        xc0 += rk[li];
+      } else if (id == r1) {
+        xa1 += rq[li];
+        xc1 += rk[li];
       }
     }
 #pragma unroll
@@ -1412,7 +1525,7 @@ __device__ __forceinline__ void quad_rows(const KParams &p, const QTok<D> &x, co
       const int row = t ? r1 : r0;
       const float yq = t ? yq1 : yq0, yk = t ? yk1 : yk0;
       const float xc = t ? xc1 : xc0, xa = t ? xa1 : xa0;
-      const float dt = beta * (__bfloat162float(sv[row]) - yk - xc);
+      const float dt = beta * (r.v(rb) - yk - xc);
       const float o = fmaf(ann, dt, yq + xa);
       st_out(p.out, static_cast<size_t>(tile) * D + row, o, p.out_bf16);
       p.buf_d[(static_cast<size_t>(tile) * p.W + n) * D + row] = dt;
@@ -1929,38 +2042,46 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
       uint8_t *slot = smem + st * slot_bytes;
       QTok<D> &x = s.u.qt[quad][li & 1];
       const int tl = s.tl_tile[e], ne = s.tl_n[e];
-      // the first row block's codes, fetched before the barrier
-      uint4 A0[2][2];
-      {
-        const int r0 = 32 * w + (lane >> 2), t = lane & 3;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          A0[0][h] = *reinterpret_cast<const uint4 *>(slot + r0 * D + frag_col(h, t, 0));
-          A0[1][h] = *reinterpret_cast<const uint4 *>(slot + (r0 + 8) * D + frag_col(h, t, 0));
-        }
-      }
       quad_channel<D, KDA>(p, x, slot, tl, ne, s.tl_coord[e], s.tl_a[e], w, ok);
-      // the quad's one barrier per tile; it also tells every warp whether any
-      // thread's wait expired, so that the quad leaves the loop together
-      if (quad_bar_any(quad, !ok)) {
-        qabort = true;
-        break;
-      }
-      quad_rows<D, KDA>(p, x, slot, tl, ne, s.tl_b[e], w, A0);
-      if (w == 0 && lane == 0) p.buf_n[tl] = ne + 1;
-      // This warp is done with the slot: order its generic-proxy accesses
-      // before the bulk copy that refills it.
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence_block();
-        if (atomicAdd(&s.done[st], 1) == 3) {
-          s.done[st] = 0;
-          __threadfence_block();
-          if (e + kStages < count) issue(st, e + kStages);
+      if constexpr (TR::kEarlyRelease) {
+        // everything the rows need from the slot goes to registers now, so
+        // that the slot is refilled while the rows are computed
+        RegRows rg;
+        quad_rows_load<D, KDA>(p, slot, ne, w, rg.r);
+        // This warp's reads of the slot are done: order them before the bulk
+        // copy that refills it.
+        fence_proxy_async();
+        // the quad's one barrier per tile; it also tells every warp whether
+        // any thread's wait expired, so that the quad leaves the loop together
+        if (quad_bar_any(quad, !ok)) {
+          qabort = true;
+          break;
         }
+        if (w == 0 && lane == 0 && e + kStages < count) issue(st, e + kStages);
+        quad_rows<D, KDA>(p, x, rg, tl, ne, s.tl_b[e], w);
+        if (w == 0 && lane == 0) p.buf_n[tl] = ne + 1;
+      } else {
+        if (quad_bar_any(quad, !ok)) {
+          qabort = true;
+          break;
+        }
+        quad_rows<D, KDA>(p, x, SlotRows<D, KDA>(p, slot, ne, w), tl, ne, s.tl_b[e], w);
+        if (w == 0 && lane == 0) p.buf_n[tl] = ne + 1;
+        // This warp is done with the slot: order its generic-proxy accesses
+        // before the bulk copy that refills it; the quad's last warp to get
+        // here issues that copy.
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence_block();
+          if (atomicAdd(&s.done[st], 1) == 3) {
+            s.done[st] = 0;
+            __threadfence_block();
+            if (e + kStages < count) issue(st, e + kStages);
+          }
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
     aborted = __syncthreads_or(qabort) != 0;
     i = P;
