@@ -60,7 +60,21 @@ WORKLOADS = {"qwen35_9b_gdn": wl.QWEN35_9B_GDN, "kimi_linear_kda": wl.KIMI_LINEA
 DEFAULT_WORKLOAD = "kimi_linear_kda"
 # the other workloads the default line reports as sub-objects, with the layer
 # count each cycles (enough to keep the working set above L2)
-OTHER_WORKLOADS = (("qwen35_9b_gdn", 8), ("gdn_sweep_b1024", 2), ("ragged_gdn", 4))
+OTHER_WORKLOADS = (("qwen35_9b_gdn", 8), ("ragged_gdn", 4))
+
+
+def sweep_layers(w: wl.Workload) -> int:
+    """Layers cycled at a sweep point: enough for a working set of four times
+    the L2 where 16 layers suffice, else 16 (the line then says it is partly
+    L2-resident)."""
+    per_layer = working_set_bytes(w, 1)
+    return int(min(16, max(2, math.ceil(4 * L2_BYTES / per_layer))))
+
+
+def sweep_steps(w: wl.Workload) -> int:
+    """Timed steps at a sweep point: fewer for larger batches, so that every
+    point takes a similar time."""
+    return int(min(200, max(10, round(200 * 2048 / w.tiles))))
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = [os.path.join(ROOT, "recurrent_state_quantization_decode_b200", "csrc", f)
                   for f in ("lq_decode.cu", "lq_internal.h")]
@@ -429,13 +443,24 @@ def whole_job_rate(units_per_step: int, world: int, steps: int, ms_max: float) -
 
 
 PREFILL_TOKENS = 256
+PREFILL_CHUNK = 16  # tokens per chunk of the WY-form prefill
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # SMs x fp32 lanes x 2 flops x max clock
+TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 / bf16 tensor rates
+
+
+def prefill_tensor_flops_per_token(d: int) -> float:
+    """Tensor-path flops of the chunked prefill per tile-token: S0 Kg^T and
+    S0 Qg^T (2 x 2 C d^2 per chunk of C tokens) and the rank-C state update
+    (2 C d^2), each run as three tf32 products (hi/lo split): 18 d^2."""
+    return 3.0 * (4.0 + 2.0) * d * d
 
 
 def prefill_measure(B, w: wl.Workload, ly, stream, device, world: int) -> dict:
     """lq_prefill of one layer's tiles over a PREFILL_TOKENS-token prompt
-    (seeded inputs), CUDA-event timed after one warm-up run.  Flops count the
-    exact recurrence's 7 d^2 per tile-token (decay, S k, update, S q)."""
+    (seeded inputs), CUDA-event timed after one warm-up run.  The roofline
+    counts the tensor-path products of the chunked form against the tf32
+    peak (the measured bf16 peak times the nominal tf32/bf16 ratio); the exact
+    recurrence's 7 d^2 flops per tile-token are given as context."""
     import torch
 
     T = PREFILL_TOKENS
@@ -464,13 +489,25 @@ def prefill_measure(B, w: wl.Workload, ly, stream, device, world: int) -> dict:
     torch.cuda.synchronize()
     ms = max_over_ranks(start.elapsed_time(end) / runs, world, device)
     tile_tokens = w.tiles * T
-    tflops = 7.0 * w.d * w.d * tile_tokens / (ms / 1e3) / 1e12
-    return {"tile_tokens_per_s": world * tile_tokens / (ms / 1e3), "ms": ms,
-            "prompt_tokens": T, "tiles": w.tiles,
-            "roofline": {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS,
-                         "unit": "TFLOP/s", "frac": tflops / FP32_ALU_TFLOPS,
-                         "peak_source": "148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"},
-            "kernel": "prefill_kernel (exact recurrence, state on chip, then quantizer)"}
+    sec = ms / 1e3
+    exact = 7.0 * w.d * w.d * tile_tokens / sec / 1e12
+    tensor = prefill_tensor_flops_per_token(w.d) * tile_tokens / sec / 1e12
+    try:
+        bf16 = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"])
+        src = "measured bf16 x nominal tf32/bf16 ratio (1.1 / 2.25)"
+    except (OSError, ValueError, KeyError):
+        bf16, src = 1590.0, "fallback bf16 x nominal tf32/bf16 ratio (1.1 / 2.25)"
+    peak = bf16 * TF32_PER_BF16
+    return {"tile_tokens_per_s": world * tile_tokens / sec, "ms": ms,
+            "prompt_tokens": T, "tiles": w.tiles, "chunk_tokens": PREFILL_CHUNK,
+            "roofline": {"bound": "tensor", "achieved": tensor, "peak": peak,
+                         "unit": "TFLOP/s", "frac": tensor / peak, "peak_source": src,
+                         "flops": "18 d^2 per tile-token: S0 Kg^T, S0 Qg^T and the rank-16 "
+                                  "update, three tf32 products each"},
+            "exact_recurrence": {"tflops": exact, "fp32_alu_peak": FP32_ALU_TFLOPS,
+                                 "frac_of_fp32_alu": exact / FP32_ALU_TFLOPS,
+                                 "flops": "7 d^2 per tile-token"},
+            "kernel": "chunk_prefill_kernel (WY form in 16-token chunks, then quantizer)"}
 
 
 def load_peaks() -> tuple[float, str]:
@@ -711,6 +748,23 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
                                              phases=key == "ragged_gdn")
             torch.cuda.synchronize()
             torch.cuda.empty_cache()
+        # the bandwidth sweep: int8 and fp32 states side by side, batch 8 .. 1024
+        sweep = []
+        for b in wl.SWEEP_BATCHES:
+            sw = wl.sweep_workload(b)
+            with nvtx(f"sweep point batch {b}"):
+                r = measure_decode(B, sw, f"gdn_sweep_b{b}", sweep_layers(sw), sweep_steps(sw),
+                                   args.warmup, stream, device, world, rank)
+            sweep.append({"batch": b, "tiles": sw.tiles, "int8_state": r["value"],
+                          "fp32_state": r["fp32_state"]["value"],
+                          "speedup_vs_fp32_state": r["speedup_vs_fp32_state"],
+                          "int8_hbm_gbs": r["hbm_gbs"], "fp32_hbm_gbs": r["fp32_state"]["hbm_gbs"],
+                          "roofline_frac": r["roofline"]["frac"], "steps": r["steps"],
+                          "layers_cycled": r["config"]["layers_cycled"],
+                          "l2": r["config"]["l2"]})
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        others["gdn_bandwidth_sweep"] = {"unit": UNIT, "points": sweep}
 
     if rank != 0:
         return

@@ -38,8 +38,8 @@
  *  buf_k    [B][Hk][W][d] keys of the buffered tokens, in the input dtype
  *           (lossless: they are the inputs themselves).
  *  buf_d    [B][Hv][W][d] fp32 deltas d_i of the buffered tokens.
- *  buf_g    [B][Hv][16] (GDN, the first W used) or [B][Hv][W][d] (KDA)
- *           fp32 gates alpha_i.
+ *  buf_g    [B][Hv][16] (GDN with W <= 16; [B][Hv][32] for W > 16; the
+ *           first W used) or [B][Hv][W][d] (KDA) fp32 gates alpha_i.
  *  buf_n    [B][Hv] int32 tokens buffered in the current window (0..W-1
  *           between calls).
  *  err      one int32 device error word (bit 0: a corrupt buf_n was seen,
@@ -56,7 +56,7 @@
  *    default).
  *  - Argument errors are detected on the host before anything is launched,
  *    and reported synchronously: LQ_ERR_INVALID_ARG (null pointer, bad
- *    shape), LQ_ERR_UNSUPPORTED (d not in {32, 64, 128}, W not in 1..16,
+ *    shape), LQ_ERR_UNSUPPORTED (d not in {32, 64, 128}, W not in 1..32,
  *    K not in 0..8, smooth not in {0, 0.5, 1}), LQ_ERR_MISALIGNED (records,
  *    buffers or the fp32 state not 16-byte aligned).  A failed launch returns
  *    LQ_ERR_CUDA.  Work is asynchronous on `stream`.
@@ -96,7 +96,7 @@ typedef struct {
   int32_t num_k_heads; /* Hk key/query heads, 1..2048 */
   int32_t num_v_heads; /* Hv >= 1 value heads, a multiple of Hk */
   int32_t d;           /* d_k = d_v = d, one of 32, 64, 128 */
-  int32_t window;      /* W tokens per quantization window, 1..16 (16 on the pages) */
+  int32_t window;      /* W tokens per quantization window, 1..32 (16 on the pages) */
   int32_t n_comp;      /* K compensator lines per tile, 0..8 (4 on the pages) */
   int32_t gate;        /* lq_gate: LQ_GATE_SCALAR (GDN) or LQ_GATE_DIAG (KDA) */
   int32_t in_dtype;    /* lq_dtype of q, k, v */
@@ -159,13 +159,20 @@ lq_status lq_state_init(const lq_config *cfg, const float *S0, const lq_state *s
  * 16-byte aligned; NULL = zero states), it runs the exact recurrence in fp32
  * for t = 0 .. T-1:
  *   S <- S diag(alpha_t); S <- S + beta_t (v_t - S k_t) k_t^T; o_t = S q_t
- * token by token with the state held on chip (not the chunked form), writes
- * the T outputs (out: [T][B][Hv][d] in out_dtype; NULL = none), and then
- * quantizes S_T into the record exactly as lq_state_init does (buffers empty,
- * buf_n = 0).  Inputs are token-major: q, k [T][B][Hk][d], v [T][B][Hv][d]
- * (in_dtype), alpha [T][B][Hv] (GDN) or [T][B][Hv][d] (KDA), beta
- * [T][B][Hv], fp32.  T >= 0 (T = 0 quantizes S0).  mask: nullable [B] int32;
- * masked-off sequences are left untouched. */
+ * with the state held on chip, writes the T outputs (out: [T][B][Hv][d] in
+ * out_dtype; NULL = none), and then quantizes S_T into the record exactly as
+ * lq_state_init does (buffers empty, buf_n = 0).  Inputs are token-major:
+ * q, k [T][B][Hk][d], v [T][B][Hv][d] (in_dtype), alpha [T][B][Hv] (GDN) or
+ * [T][B][Hv][d] (KDA), beta [T][B][Hv], fp32.  T >= 0 (T = 0 quantizes S0).
+ * mask: nullable [B] int32; masked-off sequences are left untouched.
+ * The recurrence runs in chunks of 16 tokens in its WY form: with cumulative
+ * gates g_t inside a chunk, Kg = K o g, Kh = K / g, Qg = Q o g,
+ *   U = (I + strict_lower(diag(beta) Kg Kh^T))^-1 diag(beta) (V - Kg S^T),
+ *   O = Qg S^T + lower(Qg Kh^T) U,  S <- S diag(g_last) + U^T (Kh o g_last),
+ * equal to the token loop in exact arithmetic; the products with the state
+ * run on the tensor cores at about fp32 accuracy.  Kh divides by the gates,
+ * so the product of any 16 consecutive gates must stay a normal fp32 number
+ * (above 1.2e-38). */
 lq_status lq_prefill(const lq_config *cfg, const void *q, const void *k, const void *v,
                      const float *alpha, const float *beta, int32_t T, const float *S0,
                      const lq_state *st, void *out, const int32_t *mask, void *stream);
@@ -185,6 +192,24 @@ lq_status lq_prefill(const lq_config *cfg, const void *q, const void *k, const v
 lq_status lq_decode_step(const lq_config *cfg, const void *q, const void *k, const void *v,
                          const float *alpha, const float *beta, const lq_state *st, void *out,
                          const int32_t *active, void *stream);
+
+/* ntok consecutive decode tokens for every tile in ONE launch, e.g. the
+ * verify step of speculative decoding: the result is that of ntok calls of
+ * lq_decode_step with the same active mask, folds at window boundaries
+ * included.  Inside a window the stored record is fixed and each token only
+ * reads it (zhichai.net summary, "Abstract (translated)" item 1), so the
+ * launch reads each record once for all its tokens instead of once per token.
+ * Inputs and outputs are token-major, each token laid out as for
+ * lq_decode_step: q, k [ntok][B][Hk][d], v [ntok][B][Hv][d] in_dtype (16-byte
+ * aligned); alpha [ntok][B][Hv] (GDN) or [ntok][B][Hv][d] (KDA, 16-byte
+ * aligned); beta [ntok][B][Hv] fp32; out [ntok][B][Hv][d] out_dtype.
+ * ntok >= 0 (0 does nothing).  Rejected drafts are dropped afterwards with
+ * lq_window_rewind.  One CTA per tile keeps the tile in shared memory for all
+ * its tokens; this call also serves every decode step of windows longer than
+ * 16 tokens. */
+lq_status lq_decode_tokens(const lq_config *cfg, int32_t ntok, const void *q, const void *k,
+                           const void *v, const float *alpha, const float *beta,
+                           const lq_state *st, void *out, const int32_t *active, void *stream);
 
 /* lq_decode_step with the token's inputs and output in HOST memory: moves
  * q, k, v, alpha, beta to `staging` (device, layout.host_staging_bytes,

@@ -35,7 +35,7 @@ EXPORTED = ("lq_version", "lq_status_string", "lq_state_layout", "lq_state_bytes
             "lq_decode_step_host_noalloc", "lq_window_flush",
             "lq_fp32_decode_step", "lq_state_dequantize", "lq_get_last_error",
             "lq_test_decode_step_timeout", "lq_prefill", "lq_checkpoint_save",
-            "lq_checkpoint_restore", "lq_window_rewind")
+            "lq_checkpoint_restore", "lq_window_rewind", "lq_decode_tokens")
 
 
 class lq_config(ctypes.Structure):
@@ -83,6 +83,8 @@ _sig = {
     "lq_checkpoint_save": ([_CFG, _ST, _P, _P, ctypes.c_int32, _P], ctypes.c_int),
     "lq_checkpoint_restore": ([_CFG, _P, ctypes.c_int32, _P, _ST, _P], ctypes.c_int),
     "lq_window_rewind": ([_CFG, _ST, _P, _P], ctypes.c_int),
+    "lq_decode_tokens": ([_CFG, ctypes.c_int32, _P, _P, _P, _P, _P, _ST, _P, _P, _P],
+                         ctypes.c_int),
 }
 for _name, (_args, _res) in _sig.items():
     _f = getattr(_lib, _name)
@@ -178,6 +180,15 @@ def lq_decode_step(cfg, q, k, v, alpha, beta, state: lq_state, out, active=None,
     _check(_lib.lq_decode_step(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
                                _ptr(beta), ctypes.byref(state), _ptr(out), _ptr(active),
                                _stream(stream)), "lq_decode_step")
+
+
+def lq_decode_tokens(cfg, ntok: int, q, k, v, alpha, beta, state: lq_state, out, active=None,
+                     stream=None) -> None:
+    """ntok consecutive decode tokens in one launch (token-major inputs and
+    outputs, each token laid out as for lq_decode_step)."""
+    _check(_lib.lq_decode_tokens(ctypes.byref(cfg), ctypes.c_int32(ntok), _ptr(q), _ptr(k),
+                                 _ptr(v), _ptr(alpha), _ptr(beta), ctypes.byref(state),
+                                 _ptr(out), _ptr(active), _stream(stream)), "lq_decode_tokens")
 
 
 def lq_prefill(cfg, q, k, v, alpha, beta, T: int, S0, state: lq_state, out=None, mask=None,

@@ -34,7 +34,7 @@ lq_status check_config(const lq_config *c) {
   if (c->in_dtype != LQ_DTYPE_F32 && c->in_dtype != LQ_DTYPE_BF16) return LQ_ERR_INVALID_ARG;
   if (c->out_dtype != LQ_DTYPE_F32 && c->out_dtype != LQ_DTYPE_BF16) return LQ_ERR_INVALID_ARG;
   if (c->d != 32 && c->d != 64 && c->d != 128) return LQ_ERR_UNSUPPORTED;
-  if (c->window < 1 || c->window > lq::kMaxWindow) return LQ_ERR_UNSUPPORTED;
+  if (c->window < 1 || c->window > lq::kMaxWindowLong) return LQ_ERR_UNSUPPORTED;
   if (c->n_comp < 0 || c->n_comp > lq::kMaxComp) return LQ_ERR_UNSUPPORTED;
   if (!(c->smooth == 0.0f || c->smooth == 0.5f || c->smooth == 1.0f)) return LQ_ERR_UNSUPPORTED;
   // tiles are indexed with 32-bit ints; the decode kernel packs (sequence,
@@ -82,6 +82,8 @@ KParams make_params(const lq_config *c, const lq_state *st) {
   p.smooth = c->smooth == 0.0f ? 0 : (c->smooth == 0.5f ? 1 : 2);
   p.L = lq::record_layout(c->d, c->n_comp);
   p.wait_limit = lq::kWaitLimitDefault;
+  p.gstride = lq::gdn_gate_stride(c->window);
+  p.ntok = 1;
   if (st != nullptr) {
     p.records = static_cast<uint8_t *>(st->records);
     p.buf_k = st->buf_k;
@@ -156,7 +158,8 @@ lq_status lq_state_layout(const lq_config *cfg, lq_layout *out) {
   out->records_bytes = tiles * L.bytes;
   out->buf_k_bytes = B * Hk * W * d * in_size(cfg);
   out->buf_d_bytes = tiles * W * d * 4;
-  out->buf_g_bytes = cfg->gate == LQ_GATE_DIAG ? tiles * W * d * 4 : tiles * lq::kGdnGateStride * 4;
+  out->buf_g_bytes = cfg->gate == LQ_GATE_DIAG ? tiles * W * d * 4
+                                                : tiles * lq::gdn_gate_stride(cfg->window) * 4;
   out->buf_n_bytes = tiles * 4;
   out->err_bytes = 4;
   out->fp32_state_bytes = tiles * d * d * 4;
@@ -205,6 +208,28 @@ lq_status lq_decode_step(const lq_config *cfg, const void *q, const void *k, con
   p.out = out;
   p.mask = active;
   return from_cuda(lq::launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
+lq_status lq_decode_tokens(const lq_config *cfg, int32_t ntok, const void *q, const void *k,
+                           const void *v, const float *alpha, const float *beta,
+                           const lq_state *st, void *out, const int32_t *active, void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if (ntok < 0) return LQ_ERR_INVALID_ARG;
+  if (ntok == 0 || cfg->batch == 0) return LQ_OK;
+  if ((s = check_io(cfg, q, k, v, alpha, beta, out)) != LQ_OK) return s;
+  if (!aligned_to(active, 4)) return LQ_ERR_MISALIGNED;
+  KParams p = make_params(cfg, st);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.out = out;
+  p.mask = active;
+  p.ntok = ntok;
+  return from_cuda(lq::launch_decode_tokens(p, static_cast<cudaStream_t>(stream)));
 }
 
 lq_status lq_prefill(const lq_config *cfg, const void *q, const void *k, const void *v,

@@ -42,8 +42,12 @@
 //    path with each operand split into hi and lo parts, whose accumulator
 //    fragment is that layout.  The quantizer (compensator lines, smoothing,
 //    per-row int8) then runs on it.
-//  * prefill_kernel runs the exact recurrence over a prompt with the state in
-//    the same registers and ends in the same quantizer.
+//  * chunk_prefill_kernel runs the exact recurrence over a prompt in 16-token
+//    chunks of its WY form, the products with the state on the tf32 tensor
+//    path with the state itself in the codes' fragment layout, and ends in the
+//    same quantizer.
+//  * tokens_kernel decodes several tokens per tile in one launch (one CTA per
+//    tile), and serves windows longer than 16 tokens.
 //
 // Fragment layout: warp w < D/16 owns state rows 16w..16w+15; lane (g = lane/4,
 // t = lane%4) owns rows 16w+g and 16w+g+8 and, in every 64-column span h, the
@@ -105,12 +109,12 @@ __device__ __forceinline__ bool chunk_valid(int t) {
 // One tile's staged data (a ring slot): the record, the buffered tokens and the
 // token's inputs, each at a 16-byte aligned offset.  The record area has the
 // record's actual size (it depends on K).
-template <int D, bool BF16, bool KDA>
+template <int D, bool BF16, bool KDA, int WM = kMaxWindow>
 struct SL {
   static constexpr int IB = BF16 ? 2 : 4;
-  static constexpr int BD = kMaxWindow * D * 4;                  // fp32 [W][D]
-  static constexpr int BK = kMaxWindow * D * IB;                 // in dtype [W][D]
-  static constexpr int BG = KDA ? kMaxWindow * D * 4 : kGdnGateStride * 4;
+  static constexpr int BD = WM * D * 4;                  // fp32 [WM][D]
+  static constexpr int BK = WM * D * IB;                 // in dtype [WM][D]
+  static constexpr int BG = KDA ? WM * D * 4 : WM * 4;   // KDA [WM][D]; GDN up to WM gates
   static constexpr int TAIL = BD + BK + BG + 3 * D * IB + (KDA ? D * 4 : 0);
   // quantizer scratch aliased over the codes once they are in registers
   static constexpr int QS_COLPART = 0;                           // fp64 [D/16][D]
@@ -133,17 +137,17 @@ struct SL {
 // coefficients on the bf16 tensor path (fast) and, at d = 128, keeps the
 // fold's scaled keys over the staged codes instead of in the scratch, which
 // leaves room for three ring slots at two CTAs per SM.
-template <int D, bool BF16, bool KDA>
+template <int D, bool BF16, bool KDA, int WM = kMaxWindow>
 struct DecodeTraits {
   // plain tokens (no fold) of d = 128 tiles with bf16 inputs run on the quad
   // path: four warps per tile, two tiles at once per CTA
-  static constexpr bool kQuad = BF16 && D == 128;
+  static constexpr bool kQuad = BF16 && D == 128 && WM == kMaxWindow;
   // with one ring slot per quad (KDA), the quad releases its slot at its
   // barrier, after loading the row-phase operands into registers
   static constexpr bool kEarlyRelease = kQuad && KDA;
   static_assert(kEarlyRelease == (kQuad && KDA), "one ring slot per quad only on KDA");
-  static constexpr bool kFast = BF16 && !KDA;
-  static constexpr bool kKtOverCodes = kFast && kMaxWindow * FG<D>::PADW * 4 <= D * D;
+  static constexpr bool kFast = BF16 && !KDA && WM == kMaxWindow;
+  static constexpr bool kKtOverCodes = kFast && WM * FG<D>::PADW * 4 <= D * D;
   static constexpr int kStages = kFast ? 3 : 2;
   static constexpr int kTok = kFast ? 2 : 1;  // per-token scratch buffers
   // the fold's rank-W update on the tf32 tensor path (3 products per term)
@@ -172,18 +176,18 @@ __device__ __forceinline__ int kt_mma_pos(int c) {
 
 // The scaled-key array lives in the scratch unless the decode kernel keeps it
 // over the staged codes (GDN with bf16 inputs).
-template <int D, bool KT>
+template <int D, bool KT, int WM = kMaxWindow>
 struct KtArea {
-  alignas(16) float kt[kMaxWindow][FG<D>::PADW];  // keys times decay ratio to the last token
+  alignas(16) float kt[WM][FG<D>::PADW];  // keys times decay ratio to the last token
 };
-template <int D>
-struct KtArea<D, false> {};
+template <int D, int WM>
+struct KtArea<D, false, WM> {};
 
 // Per-token values that the row phase reads: written before the tile's CTA
 // barrier, read after it.  The decode kernel for GDN with bf16 inputs keeps two
 // of these, so that one tile's per-channel work can overlap the previous
 // tile's row phase.
-template <int D>
+template <int D, int WM = kMaxWindow>
 struct Tok {
   alignas(16) float qf[D];
   alignas(16) float kf[D];
@@ -191,10 +195,10 @@ struct Tok {
   alignas(16) float G[D];                          // window gate Gamma per key channel
   alignas(16) float mG[FG<D>::PADW];               // m o Gamma
   alignas(16) int8_t dig[8][FG<D>::DIGW];          // digits: rows 0-3 of x_q, 4-7 of x_k
-  float cc[kMaxWindow + 1];
-  float aa[kMaxWindow + 1];
+  float cc[WM + 1];
+  float aa[WM + 1];
   float cpart[kMaxComp][kWarps][2];  // per-warp partial row-compensator dots
-  float rho[kMaxWindow + 1];         // scalar decay ratios (GDN)
+  float rho[WM + 1];                 // scalar decay ratios (GDN)
   float xmax[2][kWarps];
   float xscale[2][4];  // digit scales of x_q, x_k (per int8 k-chunk on the GDN-bf16 path)
 };
@@ -214,19 +218,19 @@ struct QTok {
   float cpk[4][2 * kMaxWindow];             // KDA: per warp, partial c_s (s) and a_s (16 + s)
 };
 
-template <int D, int NT, bool Q>
+template <int D, int NT, bool Q, int WM>
 union TokArea {
-  Tok<D> tok[NT];
+  Tok<D, WM> tok[NT];
 };
-template <int D, int NT>
-union TokArea<D, NT, true> {
-  Tok<D> tok[NT];     // the whole-CTA path
-  QTok<D> qt[2][2];   // the quad path: [quad][buffer]
+template <int D, int NT, int WM>
+union TokArea<D, NT, true, WM> {
+  Tok<D, WM> tok[NT];  // the whole-CTA path
+  QTok<D> qt[2][2];    // the quad path: [quad][buffer]
 };
 
-template <int D, bool KT, int NT = 1, bool Q = false>
-struct Scratch : KtArea<D, KT> {
-  TokArea<D, NT, Q> u;
+template <int D, bool KT, int NT = 1, bool Q = false, int WM = kMaxWindow>
+struct Scratch : KtArea<D, KT, WM> {
+  TokArea<D, NT, Q, WM> u;
   alignas(16) float invm[FG<D>::PADW];             // 1 / m (new smoothing factors)
   alignas(16) float line[D];                       // the compensator line being extracted
   alignas(16) double rowE[D];
@@ -518,13 +522,80 @@ __device__ __forceinline__ void at_slot(float2 (&S)[2][NSPAN][8], int h, int e, 
 #undef LQ_SPAN
 #undef LQ_SLOT
 
+// S += sum_{s < nent} d_s kt_s^T for the thread's block on the tf32 tensor
+// path: A = d (16 rows x 8 tokens, rows [s][D] in bd), B = scaled keys (8
+// tokens x 8 columns) in the layout of kt_mma_pos (rows of kt_mma_stride);
+// each operand is split into hi and lo tf32 parts and three products are
+// accumulated.  Tokens at or beyond nent (at most SMAX) contribute zero.
+template <int D, int SMAX>
+__device__ __forceinline__ void rank_update_mma(float2 (&S)[2][FG<D>::NSPAN][8], const float *bd,
+                                                const float *kt, int nent) {
+  using G = FG<D>;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int r0 = 16 * warp + g, r1 = r0 + 8;
+  constexpr int P = kt_mma_stride<D>();
+#pragma unroll
+  for (int ks = 0; ks < SMAX / 8; ++ks) {
+    if (8 * ks >= nent) break;
+    const int s0 = 8 * ks + t, s1 = s0 + 4;
+    uint32_t ah[4], al[4];
+    tf32_split(s0 < nent ? bd[s0 * D + r0] : 0.0f, ah[0], al[0]);
+    tf32_split(s0 < nent ? bd[s0 * D + r1] : 0.0f, ah[1], al[1]);
+    tf32_split(s1 < nent ? bd[s1 * D + r0] : 0.0f, ah[2], al[2]);
+    tf32_split(s1 < nent ? bd[s1 * D + r1] : 0.0f, ah[3], al[3]);
+#pragma unroll
+    for (int h = 0; h < G::NSPAN; ++h)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int pos = 64 * h + 8 * j + g;
+        uint32_t bh0, bl0, bh1, bl1;
+        tf32_split(s0 < nent ? kt[s0 * P + pos] : 0.0f, bh0, bl0);
+        tf32_split(s1 < nent ? kt[s1 * P + pos] : 0.0f, bh1, bl1);
+        mma_tf32(S[0][h][j], S[1][h][j], al[0], al[1], al[2], al[3], bh0, bh1);
+        mma_tf32(S[0][h][j], S[1][h][j], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+        mma_tf32(S[0][h][j], S[1][h][j], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+      }
+  }
+}
+
+// The same update with packed FMAs, two columns per instruction; kt rows of
+// PADW in the padded column layout (padc).
+template <int D>
+__device__ __forceinline__ void rank_update_ffma(float2 (&S)[2][FG<D>::NSPAN][8], const float *bd,
+                                                 const float *kt, int nent) {
+  using G = FG<D>;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int r0 = 16 * warp + g, r1 = r0 + 8;
+  for (int sl = 0; sl < nent; ++sl) {
+    const float2 d0 = make_float2(bd[sl * D + r0], bd[sl * D + r0]);
+    const float2 d1 = make_float2(bd[sl * D + r1], bd[sl * D + r1]);
+#pragma unroll
+    for (int h = 0; h < G::NSPAN; ++h) {
+      if (!chunk_valid<D>(t)) continue;
+      const float4 *k4 =
+          reinterpret_cast<const float4 *>(&kt[sl * G::PADW + padc(frag_col(h, t, 0))]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 k = k4[u];
+        const float2 ka = make_float2(k.x, k.y), kb = make_float2(k.z, k.w);
+        S[0][h][2 * u] = __ffma2_rn(d0, ka, S[0][h][2 * u]);
+        S[0][h][2 * u + 1] = __ffma2_rn(d0, kb, S[0][h][2 * u + 1]);
+        S[1][h][2 * u] = __ffma2_rn(d1, ka, S[1][h][2 * u]);
+        S[1][h][2 * u + 1] = __ffma2_rn(d1, kb, S[1][h][2 * u + 1]);
+      }
+    }
+  }
+}
+
 // The fp32 state of the thread's block (warps that own rows), as float2 pairs
 // along the columns:
 //   S_ij = sigma_i code_ij (m_j Gamma_j) + sum_{s < nent} d_s[i] kt_s[j]
 //          + Gamma_j * (compensator lines),
 // with kt_s = k_s o (decay ratio to the last token) in kt (rows of PADW) and m o Gamma in
 // x.mG.  rsig, rcv, rcid point at the staged record; bd at the staged deltas.
-template <int D, bool MMA = false, class SC>
+template <int D, bool MMA = false, int WM = kMaxWindow, class SC>
 __device__ __forceinline__ void build_state(const SC &x, const float *kt,
                                             const uint4 (&A)[2][FG<D>::NSPAN],
                                             const float *rsig, const float *rcv, const int *rcid,
@@ -558,54 +629,10 @@ __device__ __forceinline__ void build_state(const SC &x, const float *kt,
       for (int e2 = 0; e2 < 8; ++e2) S[0][h][e2] = S[1][h][e2] = make_float2(0.0f, 0.0f);
     }
   }
-  if constexpr (MMA) {
-    // rank-nent update on the tf32 tensor path: A = d (16 rows x 8 tokens),
-    // B = scaled keys (8 tokens x 8 columns) in the layout of kt_mma_pos;
-    // tokens at or beyond nent contribute zero
-    constexpr int P = kt_mma_stride<D>();
-#pragma unroll
-    for (int ks = 0; ks < kMaxWindow / 8; ++ks) {
-      if (8 * ks >= nent) break;
-      const int s0 = 8 * ks + t, s1 = s0 + 4;
-      uint32_t ah[4], al[4];
-      tf32_split(s0 < nent ? bd[s0 * D + r0] : 0.0f, ah[0], al[0]);
-      tf32_split(s0 < nent ? bd[s0 * D + r1] : 0.0f, ah[1], al[1]);
-      tf32_split(s1 < nent ? bd[s1 * D + r0] : 0.0f, ah[2], al[2]);
-      tf32_split(s1 < nent ? bd[s1 * D + r1] : 0.0f, ah[3], al[3]);
-#pragma unroll
-      for (int h = 0; h < G::NSPAN; ++h)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int pos = 64 * h + 8 * j + g;
-          uint32_t bh0, bl0, bh1, bl1;
-          tf32_split(s0 < nent ? kt[s0 * P + pos] : 0.0f, bh0, bl0);
-          tf32_split(s1 < nent ? kt[s1 * P + pos] : 0.0f, bh1, bl1);
-          mma_tf32(S[0][h][j], S[1][h][j], al[0], al[1], al[2], al[3], bh0, bh1);
-          mma_tf32(S[0][h][j], S[1][h][j], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
-          mma_tf32(S[0][h][j], S[1][h][j], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
-        }
-    }
-  }
-  // rank-nent update, two columns per packed FMA
-  for (int sl = 0; sl < (MMA ? 0 : nent); ++sl) {
-    const float2 d0 = make_float2(bd[sl * D + r0], bd[sl * D + r0]);
-    const float2 d1 = make_float2(bd[sl * D + r1], bd[sl * D + r1]);
-#pragma unroll
-    for (int h = 0; h < G::NSPAN; ++h) {
-      if (!chunk_valid<D>(t)) continue;
-      const float4 *k4 =
-          reinterpret_cast<const float4 *>(&kt[sl * G::PADW + padc(frag_col(h, t, 0))]);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 k = k4[u];
-        const float2 ka = make_float2(k.x, k.y), kb = make_float2(k.z, k.w);
-        S[0][h][2 * u] = __ffma2_rn(d0, ka, S[0][h][2 * u]);
-        S[0][h][2 * u + 1] = __ffma2_rn(d0, kb, S[0][h][2 * u + 1]);
-        S[1][h][2 * u] = __ffma2_rn(d1, ka, S[1][h][2 * u]);
-        S[1][h][2 * u + 1] = __ffma2_rn(d1, kb, S[1][h][2 * u + 1]);
-      }
-    }
-  }
+  if constexpr (MMA)
+    rank_update_mma<D, WM>(S, bd, kt, nent);
+  else
+    rank_update_ffma<D>(S, bd, kt, nent);
   // compensator lines, decayed by Gamma
   for (int c = 0; c < K; ++c) {
     const int id = rcid[c];
@@ -848,9 +875,13 @@ __device__ void quantize_tile(SC &s, double *colpart, float *colmax,
         }
       }
     }
+    // Row maxima of both rows, then sigma = b / 127 and 1 / sigma = 127 / b,
+    // each correctly rounded: one division per lane, lane t of a row group
+    // taking row t / 2 (sigma for even t, its inverse for odd t), shared by
+    // shuffles.  A row below FLT_MIN gets sigma = 1 and zero codes.
+    float bm[2];
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
-      const int row = rr ? r1 : r0;
       float bmax = 0.0f;
 #pragma unroll
       for (int h = 0; h < G::NSPAN; ++h) {
@@ -860,17 +891,23 @@ __device__ void quantize_tile(SC &s, double *colpart, float *colmax,
           bmax = fmaxf(bmax, fmaxf(fabsf(S[rr][h][e2].x), fabsf(S[rr][h][e2].y)));
       }
       bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, 1));
-      bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, 2));
-      float sg, inv;
-      if (bmax < FLT_MIN) {
-        sg = 1.0f;
-        inv = 0.0f;
-      } else {
-        sg = __fdiv_rn(bmax, 127.0f);
-        inv = __fdiv_rn(127.0f, bmax);
-      }
-      if (t == 0) rsig[row] = sg;
-      const float2 inv2 = make_float2(inv, inv);
+      bm[rr] = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, 2));
+    }
+    const float bsel = (t >> 1) ? bm[1] : bm[0];
+    float qd;
+    if (bsel < FLT_MIN)
+      qd = (t & 1) ? 0.0f : 1.0f;
+    else
+      qd = (t & 1) ? __fdiv_rn(127.0f, bsel) : __fdiv_rn(bsel, 127.0f);
+    const int base_lane = lane & ~3;
+    const float sgv[2] = {__shfl_sync(kFull, qd, base_lane), __shfl_sync(kFull, qd, base_lane | 2)};
+    const float invv[2] = {__shfl_sync(kFull, qd, base_lane | 1),
+                           __shfl_sync(kFull, qd, base_lane | 3)};
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int row = rr ? r1 : r0;
+      if (t == 0) rsig[row] = sgv[rr];
+      const float2 inv2 = make_float2(invv[rr], invv[rr]);
 #pragma unroll
       for (int h = 0; h < G::NSPAN; ++h) {
         if (!chunk_valid<D>(t)) continue;
@@ -1551,12 +1588,12 @@ __device__ __forceinline__ void quad_rows(const KParams &p, const QTok<D> &x, co
 //  C  every row warp: y_q, y_k for its 16 rows on the int8 tensor path, then
 //     finishes its rows (buffer sums split over the 4 lanes of a row):
 //     d_t = beta (v - y_k - sum c_s d_s), o_t = y_q + sum a_s d_s + a_t d_t.
-template <int D, bool BF16, bool KDA, class SC, class Refill>
-__device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x, uint8_t *slot,
+template <int D, bool BF16, bool KDA, int WM, class SC, class Refill>
+__device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D, WM> &x, uint8_t *slot,
                                              int tile, int n, int coord, float alpha0,
                                              float beta, Refill &&refill) {
   using G = FG<D>;
-  using L = SL<D, BF16, KDA>;
+  using L = SL<D, BF16, KDA, WM>;
   using IT = in_t<BF16>;
   constexpr int CW = (D + 31) / 32;  // channel warps
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1578,8 +1615,8 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
   const float *sa = reinterpret_cast<const float *>(slot + lay.a);
 
   // ---- Phases A and B ----
-  constexpr bool kFast = DecodeTraits<D, BF16, KDA>::kFast;
-  constexpr bool kMmaF = DecodeTraits<D, BF16, KDA>::kMmaFold;
+  constexpr bool kFast = DecodeTraits<D, BF16, KDA, WM>::kFast;
+  constexpr bool kMmaF = DecodeTraits<D, BF16, KDA, WM>::kMmaFold;
   constexpr int NCH = 2 * G::NSPAN;    // int8 MMA k-chunks (GDN-bf16: one channel warp each)
   constexpr int CWP = kFast ? 1 : CW;  // warps holding compensator partial dots
   uint4 A[2][G::NSPAN];
@@ -1594,7 +1631,7 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
                             alpha0, n,
                             ((static_cast<size_t>(b) * p.Hk + hk) * p.W + n) * D, writes_key,
                             warp);
-      if (tid == 0) p.buf_g[static_cast<size_t>(tile) * kGdnGateStride + n] = alpha0;
+      if (tid == 0) p.buf_g[static_cast<size_t>(tile) * p.gstride + n] = alpha0;
     } else if (warp == NCH) {
       coef_mma<D>(x, reinterpret_cast<const __nv_bfloat16 *>(sbk),
                   reinterpret_cast<const __nv_bfloat16 *>(sk),
@@ -1677,7 +1714,7 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
                                 reinterpret_cast<const __nv_bfloat16 *>(sq), sbg, alpha0, n);
   }
   if constexpr (!KDA) {
-    if (tid == 0) p.buf_g[static_cast<size_t>(tile) * kGdnGateStride + n] = alpha0;
+    if (tid == 0) p.buf_g[static_cast<size_t>(tile) * p.gstride + n] = alpha0;
   }
   __syncthreads();
 
@@ -1850,18 +1887,18 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
   uint4 Af[2][G::NSPAN];
   if (warp < G::NRB) load_codes<D>(codes, Af);
   const float *kt;
-  if constexpr (DecodeTraits<D, BF16, KDA>::kFast) {
+  if constexpr (DecodeTraits<D, BF16, KDA, WM>::kFast) {
     // scaled keys from the staged keys and the scalar ratios; at d = 128 they
     // go over the staged codes, which are now in registers
     float *ktw;
-    if constexpr (DecodeTraits<D, BF16, KDA>::kKtOverCodes) {
+    if constexpr (DecodeTraits<D, BF16, KDA, WM>::kKtOverCodes) {
       __syncthreads();
       ktw = reinterpret_cast<float *>(slot);
     } else {
       ktw = &s.kt[0][0];
     }
     if (tid < D) {
-      if constexpr (DecodeTraits<D, BF16, KDA>::kMmaFold) {
+      if constexpr (DecodeTraits<D, BF16, KDA, WM>::kMmaFold) {
         constexpr int P = kt_mma_stride<D>();
         const int pos = kt_mma_pos(tid);
         for (int sl = 0; sl < n; ++sl)
@@ -1879,7 +1916,7 @@ __device__ __forceinline__ bool process_tile(const KParams &p, SC &s, Tok<D> &x,
     kt = &s.kt[0][0];
   }
   if (warp < G::NRB)
-    build_state<D, DecodeTraits<D, BF16, KDA>::kMmaFold>(x, kt, Af, rsig, rcv, rcid, sbd, n + 1,
+    build_state<D, DecodeTraits<D, BF16, KDA, WM>::kMmaFold, WM>(x, kt, Af, rsig, rcv, rcid, sbd, n + 1,
                                                         p.K, S);
   __syncthreads();  // the staged codes and keys are now free for the quantizer's scratch
   quantize_tile<D>(s, reinterpret_cast<double *>(slot + L::QS_COLPART),
@@ -2170,9 +2207,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
 
 // Loads a tile's record and n buffered tokens into a slot with plain 16-byte
 // loads (the whole CTA).
-template <int D, bool BF16, bool KDA>
+template <int D, bool BF16, bool KDA, int WM = kMaxWindow>
 __device__ __forceinline__ void load_slot(const KParams &p, uint8_t *slot, int tile, int n) {
-  using L = SL<D, BF16, KDA>;
+  using L = SL<D, BF16, KDA, WM>;
   const L lay(p.L.bytes);
   const int b = tile / p.Hv, h = tile - b * p.Hv, hk = h / (p.Hv / p.Hk);
   auto copy = [&](uint8_t *dst, const void *src, int bytes) {
@@ -2188,22 +2225,22 @@ __device__ __forceinline__ void load_slot(const KParams &p, uint8_t *slot, int t
          n * D * L::IB);
     if (KDA) copy(slot + lay.bg, p.buf_g + static_cast<size_t>(tile) * p.W * D, n * D * 4);
   }
-  if (!KDA) copy(slot + lay.bg, p.buf_g + static_cast<size_t>(tile) * kGdnGateStride,
-                 kGdnGateStride * 4);
+  if (!KDA) copy(slot + lay.bg, p.buf_g + static_cast<size_t>(tile) * p.gstride, p.gstride * 4);
 }
 
 // MODE 0: flush selected tiles with 0 < n < W.  MODE 1: write the fp32 state
 // (the window base, or the current state with include_buffer).
-template <int D, bool BF16, bool KDA, int MODE>
+template <int D, bool BF16, bool KDA, int MODE, int WM>
 __global__ void __launch_bounds__(kThreads) fold_kernel(const KParams p) {
   using G = FG<D>;
-  using L = SL<D, BF16, KDA>;
+  using L = SL<D, BF16, KDA, WM>;
   using IT = in_t<BF16>;
+  using SC = Scratch<D, true, 1, false, WM>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t *slot = smem;
   const L lay(p.L.bytes);
-  Scratch<D, true> &s = *reinterpret_cast<Scratch<D, true> *>(smem + lay.bytes);
-  Tok<D> &x = s.u.tok[0];
+  SC &s = *reinterpret_cast<SC *>(smem + lay.bytes);
+  Tok<D, WM> &x = s.u.tok[0];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int tile = blockIdx.x;
@@ -2216,7 +2253,7 @@ __global__ void __launch_bounds__(kThreads) fold_kernel(const KParams p) {
   }
   if (MODE == 0 && n == 0) return;
   if (MODE == 1 && !p.include_buffer) n = 0;
-  load_slot<D, BF16, KDA>(p, slot, tile, n);
+  load_slot<D, BF16, KDA, WM>(p, slot, tile, n);
   __syncthreads();
   const float *rsig = reinterpret_cast<const float *>(slot + p.L.off_sig);
   const float *rm = reinterpret_cast<const float *>(slot + p.L.off_m);
@@ -2240,7 +2277,7 @@ __global__ void __launch_bounds__(kThreads) fold_kernel(const KParams p) {
   if (warp < G::NRB) {
     uint4 A[2][G::NSPAN];
     load_codes<D>(slot, A);
-    build_state<D>(x, &s.kt[0][0], A, rsig, rcv, rcid, sbd, n, p.K, S);
+    build_state<D, false, WM>(x, &s.kt[0][0], A, rsig, rcv, rcid, sbd, n, p.K, S);
   }
   if constexpr (MODE == 0) {
     __syncthreads();
@@ -2263,6 +2300,80 @@ __global__ void __launch_bounds__(kThreads) fold_kernel(const KParams p) {
           row[u] = make_float4(S[rr][hh][2 * u].x, S[rr][hh][2 * u].y, S[rr][hh][2 * u + 1].x,
                                S[rr][hh][2 * u + 1].y);
       }
+  }
+}
+
+// Decode of p.ntok consecutive tokens per tile in one launch (a speculative
+// verify step, or every step of a window longer than kMaxWindow tokens).  One
+// CTA per tile runs the whole-CTA token path token after token with the tile
+// kept in shared memory: the record and the buffered tokens are loaded once,
+// each token's inputs are staged, its key and gate join the staged buffer
+// (process_tile stores its d_t there), and a fold, which writes the new record
+// to global memory, is followed by loading that record.  The result equals
+// p.ntok launches of the decode step on the same inputs.  Inputs and outputs
+// are token-major: token i of q sits at q + i * B * Hk * D, and so on.
+template <int D, bool BF16, bool KDA>
+__global__ void __launch_bounds__(kThreads) tokens_kernel(const KParams p) {
+  constexpr int WM = kMaxWindowLong;
+  using L = SL<D, BF16, KDA, WM>;
+  using IT = in_t<BF16>;
+  using SC = Scratch<D, true, 1, false, WM>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t *slot = smem;
+  const L lay(p.L.bytes);
+  SC &s = *reinterpret_cast<SC *>(smem + lay.bytes);
+  const int tid = threadIdx.x;
+  const int tile = blockIdx.x;
+  const int b = tile / p.Hv, h = tile - b * p.Hv, group = p.Hv / p.Hk, hk = h / group;
+  if (p.mask != nullptr && p.mask[b] == 0) return;
+  int n = p.buf_n[tile];
+  if (n < 0 || n >= p.W) {
+    if (tid == 0) atomicOr(p.err, kErrBadPhase);
+    return;
+  }
+  const int coord = (b << 12) | (hk << 1) | ((h % group == 0) ? 1 : 0);
+  const size_t tiles = static_cast<size_t>(p.B) * p.Hv;
+  const size_t qk_tok = static_cast<size_t>(p.B) * p.Hk * D, v_tok = tiles * D;
+  auto copy = [&](uint8_t *dst, const void *src, int bytes) {
+    const uint4 *s4 = static_cast<const uint4 *>(src);
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+    for (int k = tid; k < bytes / 16; k += kThreads) d4[k] = s4[k];
+  };
+  load_slot<D, BF16, KDA, WM>(p, slot, tile, n);
+  IT *sbk = reinterpret_cast<IT *>(slot + lay.bk);
+  float *sbg = reinterpret_cast<float *>(slot + lay.bg);
+  const IT *sk = reinterpret_cast<const IT *>(slot + lay.k);
+  const float *sa = reinterpret_cast<const float *>(slot + lay.a);
+  for (int i = 0; i < p.ntok; ++i) {
+    const IT *q = static_cast<const IT *>(p.q) + i * qk_tok;
+    const IT *k = static_cast<const IT *>(p.k) + i * qk_tok;
+    const IT *v = static_cast<const IT *>(p.v) + i * v_tok;
+    const size_t qk = (static_cast<size_t>(b) * p.Hk + hk) * D;
+    copy(slot + lay.q, q + qk, D * L::IB);
+    copy(slot + lay.k, k + qk, D * L::IB);
+    copy(slot + lay.v, v + static_cast<size_t>(tile) * D, D * L::IB);
+    if (KDA) copy(slot + lay.a, p.alpha + (i * tiles + tile) * D, D * 4);
+    const float a0 = KDA ? 0.0f : p.alpha[i * tiles + tile];
+    const float b0 = p.beta[i * tiles + tile];
+    __syncthreads();
+    KParams pi = p;
+    pi.out = static_cast<uint8_t *>(p.out) + i * v_tok * (p.out_bf16 ? 2 : 4);
+    process_tile<D, BF16, KDA>(pi, s, s.u.tok[0], slot, tile, n, coord, a0, b0, [] {});
+    __syncthreads();
+    if (n + 1 == p.W) {
+      // the fold wrote the new record: bring it into the slot
+      copy(slot, p.records + static_cast<size_t>(tile) * p.L.bytes, p.L.bytes);
+      n = 0;
+    } else {
+      // token i joins the staged buffer (its d_t is there already)
+      if (tid < D) {
+        sbk[n * D + tid] = sk[tid];
+        if (KDA) sbg[n * D + tid] = sa[tid];
+      }
+      if (!KDA && tid == 0) sbg[n] = a0;
+      n += 1;
+    }
+    __syncthreads();
   }
 }
 
@@ -2306,24 +2417,59 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const KParams p) {
   if (tid == 0) p.buf_n[tile] = 0;
 }
 
-// Prefill: the exact recurrence over a prompt of T tokens with the tile's
-// fp32 state held in registers (the quantizer's fragment layout), then the
-// quantizer.  Per token: S <- S diag(alpha); y = S k; d = beta (v - y);
-// S <- S + d k^T; o = S q.  The next token's inputs are loaded while the
-// current one is computed.  One CTA per tile.
+// ---------------------------------------------------------------------------
+// Chunked prefill (WY form)
+// ---------------------------------------------------------------------------
+//
+// The exact recurrence over a prompt in chunks of kChunk tokens.  Within a
+// chunk with cumulative gates g_t (g_t = alpha_1 ... alpha_t from the chunk's
+// start; a scalar for GDN, per key channel for KDA), Kg = K o g, Kh = K / g
+// and Qg = Q o g:
+//   A   = strict lower part of diag(beta) Kg Kh^T
+//   U   = (I + A)^-1 diag(beta) (V - Kg S0^T)       (forward substitution)
+//   O   = Qg S0^T + lower part (with diagonal) of Qg Kh^T, times U
+//   S_C = S0 diag(g_C) + U^T (Kh o g_C)
+// which reproduces the token loop exactly in exact arithmetic.  The products
+// with the state (S0 Kg^T, S0 Qg^T and the rank-kChunk update) run on the tf32
+// tensor path with hi/lo splits (about fp32 accuracy), with the state itself
+// as the A operand straight from registers; the small kChunk x kChunk
+// products, the substitution and the outputs use fp32 FMAs.  Kh divides by
+// the gates: the gates' product over one chunk must stay a normal fp32 number.
+constexpr int kChunk = 16;
+static_assert(kChunk * kChunk == kThreads, "one thread per entry of a chunk's A and M");
+
+template <int D>
+struct ChunkSmem {
+  static constexpr int P = D + 2;   // rows of Qg, Kg, Kh: 8-byte aligned, at most 2-way banks
+  static constexpr int PY = D + 4;  // rows of the transposed products
+  alignas(16) float qg[kChunk][P];
+  alignas(16) float kg[kChunk][P];
+  alignas(16) float kh[kChunk][P];
+  alignas(16) float v[kChunk][D];
+  alignas(16) float yk[kChunk][PY];  // (S0 Kg^T)^T
+  alignas(16) float yq[kChunk][PY];  // (S0 Qg^T)^T
+  alignas(16) float u[kChunk][D];    // U: the d_s of the chunk's state update
+  alignas(16) float kt[kChunk][FG<D>::PADW];  // Kh o g_C in the rank update's layout
+  float amat[kChunk][kChunk + 1];
+  float mmat[kChunk][kChunk + 1];
+  float gc[D];
+  float beta[kChunk];
+};
+
 template <int D, bool BF16, bool KDA>
-__global__ void __launch_bounds__(kThreads) prefill_kernel(const KParams p) {
+__global__ void __launch_bounds__(kThreads, 2) chunk_prefill_kernel(const KParams p) {
   using G = FG<D>;
   using IT = in_t<BF16>;
+  using CS = ChunkSmem<D>;
+  constexpr bool kMma = D >= 64;  // rank update on the tensor path (its column layout needs d >= 64)
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t *qscr = smem;  // D*D bytes of quantizer scratch
-  Scratch<D, false> &s = *reinterpret_cast<Scratch<D, false> *>(smem + D * D);
-  Tok<D> &x = s.u.tok[0];
+  CS &c = *reinterpret_cast<CS *>(smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int tile = blockIdx.x;
   const int b = tile / p.Hv, h = tile - b * p.Hv, hk = h / (p.Hv / p.Hk);
   if (p.mask != nullptr && p.mask[b] == 0) return;
+  const bool rows_here = warp < G::NRB;
   const int r0 = 16 * warp + g, r1 = r0 + 8;
   float2 S[2][G::NSPAN][8];
 #pragma unroll
@@ -2332,7 +2478,7 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const KParams p) {
     for (int hh = 0; hh < G::NSPAN; ++hh)
 #pragma unroll
       for (int e2 = 0; e2 < 8; ++e2) S[rr][hh][e2] = make_float2(0.0f, 0.0f);
-  if (p.S_in != nullptr && warp < G::NRB) {
+  if (p.S_in != nullptr && rows_here) {
     const float *src = p.S_in + static_cast<size_t>(tile) * D * D;
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr)
@@ -2354,93 +2500,155 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const KParams p) {
   const size_t tokB = static_cast<size_t>(p.B);
   auto qk_at = [&](int tt) { return ((tt * tokB + b) * p.Hk + hk) * D; };
   auto hv_at = [&](int tt) { return (tt * tokB + b) * p.Hv + h; };
-  // thread j < D carries channel j of the next token's inputs
-  float nq = 0.0f, nk = 0.0f, nv = 0.0f, na = 0.0f;
-  if (tid < D && p.T > 0) {
-    nq = to_f(q[qk_at(0) + tid]);
-    nk = to_f(k[qk_at(0) + tid]);
-    nv = to_f(v[hv_at(0) * D + tid]);
-    na = KDA ? p.alpha[hv_at(0) * D + tid] : 0.0f;
-  }
-  for (int tt = 0; tt < p.T; ++tt) {
+
+  for (int t0 = 0; t0 < p.T; t0 += kChunk) {
+    const int cn = p.T - t0 < kChunk ? p.T - t0 : kChunk;
+    // Channel j: the cumulative gates and Kg, Kh, Qg; v; beta.
     if (tid < D) {
-      x.qf[tid] = nq;
-      x.kf[tid] = nk;
-      x.vf[tid] = nv;
-      if (KDA) x.G[tid] = na;
-      if (tt + 1 < p.T) {
-        nq = to_f(q[qk_at(tt + 1) + tid]);
-        nk = to_f(k[qk_at(tt + 1) + tid]);
-        nv = to_f(v[hv_at(tt + 1) * D + tid]);
-        if (KDA) na = p.alpha[hv_at(tt + 1) * D + tid];
+      const int j = tid;
+      float gcum = 1.0f;
+      for (int tt = 0; tt < kChunk; ++tt) {
+        float qv = 0.0f, kv = 0.0f, vv = 0.0f, kg = 0.0f, kh = 0.0f, qg = 0.0f;
+        if (tt < cn) {
+          gcum *= KDA ? p.alpha[hv_at(t0 + tt) * D + j] : p.alpha[hv_at(t0 + tt)];
+          qv = to_f(q[qk_at(t0 + tt) + j]);
+          kv = to_f(k[qk_at(t0 + tt) + j]);
+          vv = to_f(v[hv_at(t0 + tt) * D + j]);
+          kg = kv * gcum;
+          kh = kv / gcum;
+          qg = qv * gcum;
+        }
+        c.qg[tt][j] = qg;
+        c.kg[tt][j] = kg;
+        c.kh[tt][j] = kh;
+        c.v[tt][j] = vv;
       }
+      c.gc[j] = gcum;
+      if (j < kChunk) c.beta[j] = j < cn ? p.beta[hv_at(t0 + j)] : 0.0f;
     }
     __syncthreads();
-    if (warp < G::NRB) {
-      const float a0 = KDA ? 1.0f : p.alpha[hv_at(tt)];
-      const float beta = p.beta[hv_at(tt)];
-      float y0 = 0.0f, y1 = 0.0f;
+    // The rank update's keys Kh o g_C, and the products with the state.
+    if (tid < D) {
+      for (int tt = 0; tt < kChunk; ++tt)
+        c.kt[0][tt * (kMma ? kt_mma_stride<D>() : G::PADW) +
+                (kMma ? kt_mma_pos(tid) : padc(tid))] = c.kh[tt][tid] * c.gc[tid];
+    }
+    if (rows_here) {
+      // Y = S0 X^T for X = Kg and Qg: A = the state (rows r0, r1; k-block
+      // (h, e2) takes columns 64h + 16t' + 2e2 and + 1 of lane t'), B = X^T.
+      float2 yk[2][2], yq[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) yk[nt][0] = yk[nt][1] = yq[nt][0] = yq[nt][1] = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int hh = 0; hh < G::NSPAN; ++hh) {
-        if (!chunk_valid<D>(t)) continue;
-        const float4 *k4 = reinterpret_cast<const float4 *>(&x.kf[frag_col(hh, t, 0)]);
-        const float4 *a4 = reinterpret_cast<const float4 *>(&x.G[frag_col(hh, t, 0)]);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 kk = k4[u];
-          const float4 aa = KDA ? a4[u] : make_float4(a0, a0, a0, a0);
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const bool ok = chunk_valid<D>(t);
+          uint32_t ah[4], al[4];
+          tf32_split(ok ? S[0][hh][e2].x : 0.0f, ah[0], al[0]);
+          tf32_split(ok ? S[1][hh][e2].x : 0.0f, ah[1], al[1]);
+          tf32_split(ok ? S[0][hh][e2].y : 0.0f, ah[2], al[2]);
+          tf32_split(ok ? S[1][hh][e2].y : 0.0f, ah[3], al[3]);
+          const int col = 64 * hh + 16 * t + 2 * e2;
 #pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            float2 &sa = S[rr][hh][2 * u], &sb = S[rr][hh][2 * u + 1];
-            sa = __fmul2_rn(sa, make_float2(aa.x, aa.y));
-            sb = __fmul2_rn(sb, make_float2(aa.z, aa.w));
-            float &y = rr ? y1 : y0;
-            y = fmaf(sa.x, kk.x, y);
-            y = fmaf(sa.y, kk.y, y);
-            y = fmaf(sb.x, kk.z, y);
-            y = fmaf(sb.y, kk.w, y);
+          for (int nt = 0; nt < 2; ++nt) {
+            const int tok = 8 * nt + g;
+            const float2 xk = ok ? *reinterpret_cast<const float2 *>(&c.kg[tok][col])
+                                 : make_float2(0.0f, 0.0f);
+            const float2 xq = ok ? *reinterpret_cast<const float2 *>(&c.qg[tok][col])
+                                 : make_float2(0.0f, 0.0f);
+            uint32_t bh0, bl0, bh1, bl1;
+            tf32_split(xk.x, bh0, bl0);
+            tf32_split(xk.y, bh1, bl1);
+            mma_tf32(yk[nt][0], yk[nt][1], al[0], al[1], al[2], al[3], bh0, bh1);
+            mma_tf32(yk[nt][0], yk[nt][1], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+            mma_tf32(yk[nt][0], yk[nt][1], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+            tf32_split(xq.x, bh0, bl0);
+            tf32_split(xq.y, bh1, bl1);
+            mma_tf32(yq[nt][0], yq[nt][1], al[0], al[1], al[2], al[3], bh0, bh1);
+            mma_tf32(yq[nt][0], yq[nt][1], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+            mma_tf32(yq[nt][0], yq[nt][1], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
           }
         }
       }
-      y0 += __shfl_xor_sync(kFull, y0, 1);
-      y1 += __shfl_xor_sync(kFull, y1, 1);
-      y0 += __shfl_xor_sync(kFull, y0, 2);
-      y1 += __shfl_xor_sync(kFull, y1, 2);
-      const float d0 = beta * (x.vf[r0] - y0), d1 = beta * (x.vf[r1] - y1);
-      float o0 = 0.0f, o1 = 0.0f;
+      // accumulator: rows r0 (x, y = tokens 8nt + 2t, + 1) and r1
 #pragma unroll
-      for (int hh = 0; hh < G::NSPAN; ++hh) {
-        if (!chunk_valid<D>(t)) continue;
-        const float4 *k4 = reinterpret_cast<const float4 *>(&x.kf[frag_col(hh, t, 0)]);
-        const float4 *q4 = reinterpret_cast<const float4 *>(&x.qf[frag_col(hh, t, 0)]);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 kk = k4[u], qq = q4[u];
-#pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            const float dd = rr ? d1 : d0;
-            float2 &sa = S[rr][hh][2 * u], &sb = S[rr][hh][2 * u + 1];
-            sa = __ffma2_rn(make_float2(dd, dd), make_float2(kk.x, kk.y), sa);
-            sb = __ffma2_rn(make_float2(dd, dd), make_float2(kk.z, kk.w), sb);
-            float &o = rr ? o1 : o0;
-            o = fmaf(sa.x, qq.x, o);
-            o = fmaf(sa.y, qq.y, o);
-            o = fmaf(sb.x, qq.z, o);
-            o = fmaf(sb.y, qq.w, o);
-          }
-        }
+      for (int nt = 0; nt < 2; ++nt) {
+        const int tk = 8 * nt + 2 * t;
+        c.yk[tk][r0] = yk[nt][0].x;
+        c.yk[tk + 1][r0] = yk[nt][0].y;
+        c.yk[tk][r1] = yk[nt][1].x;
+        c.yk[tk + 1][r1] = yk[nt][1].y;
+        c.yq[tk][r0] = yq[nt][0].x;
+        c.yq[tk + 1][r0] = yq[nt][0].y;
+        c.yq[tk][r1] = yq[nt][1].x;
+        c.yq[tk + 1][r1] = yq[nt][1].y;
       }
-      o0 += __shfl_xor_sync(kFull, o0, 1);
-      o1 += __shfl_xor_sync(kFull, o1, 1);
-      o0 += __shfl_xor_sync(kFull, o0, 2);
-      o1 += __shfl_xor_sync(kFull, o1, 2);
-      if (p.out != nullptr && t == 0) {
-        st_out(p.out, static_cast<size_t>(hv_at(tt)) * D + r0, o0, p.out_bf16);
-        st_out(p.out, static_cast<size_t>(hv_at(tt)) * D + r1, o1, p.out_bf16);
+    }
+    {
+      // A_ts = beta_t Kg_t . Kh_s (s < t) and M_ts = Qg_t . Kh_s (s <= t):
+      // thread (t, s) takes one entry of each
+      const int ta = tid / kChunk, sa = tid % kChunk;
+      float dk = 0.0f, dq = 0.0f;
+#pragma unroll 8
+      for (int j = 0; j < D; j += 2) {
+        const float2 x = *reinterpret_cast<const float2 *>(&c.kh[sa][j]);
+        const float2 kk = *reinterpret_cast<const float2 *>(&c.kg[ta][j]);
+        const float2 qq = *reinterpret_cast<const float2 *>(&c.qg[ta][j]);
+        dk = fmaf(kk.x, x.x, fmaf(kk.y, x.y, dk));
+        dq = fmaf(qq.x, x.x, fmaf(qq.y, x.y, dq));
+      }
+      c.amat[ta][sa] = sa < ta ? c.beta[ta] * dk : 0.0f;
+      c.mmat[ta][sa] = sa <= ta ? dq : 0.0f;
+    }
+    __syncthreads();
+    // Value channel i: U by forward substitution, then the chunk's outputs.
+    if (tid < D) {
+      const int i = tid;
+      float uu[kChunk];
+#pragma unroll
+      for (int tt = 0; tt < kChunk; ++tt) {
+        float r = c.beta[tt] * (c.v[tt][i] - c.yk[tt][i]);
+#pragma unroll
+        for (int s2 = 0; s2 < tt; ++s2) r = fmaf(-c.amat[tt][s2], uu[s2], r);
+        uu[tt] = r;
+        c.u[tt][i] = r;
+      }
+      if (p.out != nullptr) {
+#pragma unroll
+        for (int tt = 0; tt < kChunk; ++tt) {
+          if (tt >= cn) break;
+          float o = c.yq[tt][i];
+#pragma unroll
+          for (int s2 = 0; s2 <= tt; ++s2) o = fmaf(c.mmat[tt][s2], uu[s2], o);
+          st_out(p.out, static_cast<size_t>(hv_at(t0 + tt)) * D + i, o, p.out_bf16);
+        }
       }
     }
     __syncthreads();
+    // S = S0 diag(g_C) + U^T (Kh o g_C)
+    if (rows_here) {
+#pragma unroll
+      for (int hh = 0; hh < G::NSPAN; ++hh) {
+        if (!chunk_valid<D>(t)) continue;
+        const int cb = frag_col(hh, t, 0);
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const float2 gg = make_float2(c.gc[cb + 2 * e2], c.gc[cb + 2 * e2 + 1]);
+          S[0][hh][e2] = __fmul2_rn(S[0][hh][e2], gg);
+          S[1][hh][e2] = __fmul2_rn(S[1][hh][e2], gg);
+        }
+      }
+      if constexpr (kMma)
+        rank_update_mma<D, kChunk>(S, &c.u[0][0], &c.kt[0][0], cn);
+      else
+        rank_update_ffma<D>(S, &c.u[0][0], &c.kt[0][0], cn);
+    }
+    __syncthreads();  // the chunk's arrays are free for the next chunk
   }
+  // the quantizer's scratch goes over the chunk arrays
+  uint8_t *qscr = smem;  // D*D bytes
+  Scratch<D, false> &s = *reinterpret_cast<Scratch<D, false> *>(smem + D * D);
   quantize_tile<D>(s, reinterpret_cast<double *>(qscr),
                    reinterpret_cast<float *>(qscr + G::NRB * D * 8), S,
                    p.records + static_cast<size_t>(tile) * p.L.bytes, p.L, p.K, p.smooth);
@@ -2522,16 +2730,38 @@ cudaError_t decode_t(const KParams &p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <int D, bool BF16, bool KDA, int MODE, int WM>
+cudaError_t fold_wm(const KParams &p, cudaStream_t st) {
+  static LaunchInfo cache[32][kMaxComp + 1];
+  using L = SL<D, BF16, KDA, WM>;
+  using SC = Scratch<D, true, 1, false, WM>;
+  const size_t smem = L(p.L.bytes).bytes + sizeof(SC);
+  const size_t smem_max = L(record_layout(D, kMaxComp).bytes).bytes + sizeof(SC);
+  LaunchInfo li;
+  cudaError_t e = prepare(fold_kernel<D, BF16, KDA, MODE, WM>, smem, smem_max, p.K, cache, li);
+  if (e != cudaSuccess) return e;
+  fold_kernel<D, BF16, KDA, MODE, WM><<<p.B * p.Hv, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+// Windows above kMaxWindow tokens use the longer buffer capacity.
 template <int D, bool BF16, bool KDA, int MODE>
 cudaError_t fold_t(const KParams &p, cudaStream_t st) {
+  if (p.W > kMaxWindow) return fold_wm<D, BF16, KDA, MODE, kMaxWindowLong>(p, st);
+  return fold_wm<D, BF16, KDA, MODE, kMaxWindow>(p, st);
+}
+
+template <int D, bool BF16, bool KDA>
+cudaError_t tokens_t(const KParams &p, cudaStream_t st) {
   static LaunchInfo cache[32][kMaxComp + 1];
-  using L = SL<D, BF16, KDA>;
-  const size_t smem = L(p.L.bytes).bytes + sizeof(Scratch<D, true>);
-  const size_t smem_max = L(record_layout(D, kMaxComp).bytes).bytes + sizeof(Scratch<D, true>);
+  using L = SL<D, BF16, KDA, kMaxWindowLong>;
+  using SC = Scratch<D, true, 1, false, kMaxWindowLong>;
+  const size_t smem = L(p.L.bytes).bytes + sizeof(SC);
+  const size_t smem_max = L(record_layout(D, kMaxComp).bytes).bytes + sizeof(SC);
   LaunchInfo li;
-  cudaError_t e = prepare(fold_kernel<D, BF16, KDA, MODE>, smem, smem_max, p.K, cache, li);
+  cudaError_t e = prepare(tokens_kernel<D, BF16, KDA>, smem, smem_max, p.K, cache, li);
   if (e != cudaSuccess) return e;
-  fold_kernel<D, BF16, KDA, MODE><<<p.B * p.Hv, kThreads, smem, st>>>(p);
+  tokens_kernel<D, BF16, KDA><<<p.B * p.Hv, kThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -2549,11 +2779,13 @@ cudaError_t init_t(const KParams &p, cudaStream_t st) {
 template <int D, bool BF16, bool KDA>
 cudaError_t prefill_t(const KParams &p, cudaStream_t st) {
   static LaunchInfo cache[32][kMaxComp + 1];
-  const size_t smem = D * D + sizeof(Scratch<D, false>);
+  size_t smem = sizeof(ChunkSmem<D>);
+  const size_t quant = D * D + sizeof(Scratch<D, false>);
+  if (smem < quant) smem = quant;
   LaunchInfo li;
-  cudaError_t e = prepare(prefill_kernel<D, BF16, KDA>, smem, smem, p.K, cache, li);
+  cudaError_t e = prepare(chunk_prefill_kernel<D, BF16, KDA>, smem, smem, p.K, cache, li);
   if (e != cudaSuccess) return e;
-  prefill_kernel<D, BF16, KDA><<<p.B * p.Hv, kThreads, smem, st>>>(p);
+  chunk_prefill_kernel<D, BF16, KDA><<<p.B * p.Hv, kThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -2576,7 +2808,15 @@ cudaError_t dispatch3(const KParams &p, cudaStream_t s) {
 
 template <int D, bool BF, bool KDA>
 struct DecodeF {
-  static cudaError_t run(const KParams &p, cudaStream_t s) { return decode_t<D, BF, KDA>(p, s); }
+  static cudaError_t run(const KParams &p, cudaStream_t s) {
+    // windows above kMaxWindow tokens run on the per-tile kernel
+    if (p.W > kMaxWindow) return tokens_t<D, BF, KDA>(p, s);
+    return decode_t<D, BF, KDA>(p, s);
+  }
+};
+template <int D, bool BF, bool KDA>
+struct TokensF {
+  static cudaError_t run(const KParams &p, cudaStream_t s) { return tokens_t<D, BF, KDA>(p, s); }
 };
 template <int D, bool BF, bool KDA>
 struct FlushF {
@@ -2594,6 +2834,9 @@ struct PrefillF {
 }  // namespace
 
 cudaError_t launch_decode(const KParams &p, cudaStream_t s) { return dispatch3<DecodeF>(p, s); }
+cudaError_t launch_decode_tokens(const KParams &p, cudaStream_t s) {
+  return dispatch3<TokensF>(p, s);
+}
 cudaError_t launch_flush(const KParams &p, cudaStream_t s) { return dispatch3<FlushF>(p, s); }
 cudaError_t launch_dequantize(const KParams &p, cudaStream_t s) {
   return dispatch3<DequantF>(p, s);

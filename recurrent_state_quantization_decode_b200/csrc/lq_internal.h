@@ -10,9 +10,14 @@
 
 namespace lq {
 
-constexpr int kMaxWindow = 16;  // W limit: one buffer slot per token of a window
+constexpr int kMaxWindow = 16;      // W limit of the persistent decode kernel
+constexpr int kMaxWindowLong = 32;  // W limit of the per-tile kernel (longer windows)
 constexpr int kMaxComp = 8;     // K limit
 constexpr int kGdnGateStride = 16;  // GDN gate buffer: 16 floats per tile (one 64-byte copy)
+
+// Floats per tile of the GDN gate buffer for a window of W tokens: 16 up to
+// W = 16, 32 beyond.
+inline int gdn_gate_stride(int W) { return W > kGdnGateStride ? 2 * kGdnGateStride : kGdnGateStride; }
 constexpr int kErrBadPhase = 1;     // device error bit: buf_n outside [0, W)
 constexpr int kErrTimeout = 2;      // device error bit: a bounded wait on a copy expired
 
@@ -48,6 +53,8 @@ struct KParams {
   int T;                // prefill: prompt tokens
   uint32_t wait_limit;  // decode: polls of a bounded mbarrier wait before it expires
   int withhold;         // decode, testing only: CTA 0 issues no copies for its first slot
+  int gstride;          // floats per tile of the GDN gate buffer (gdn_gate_stride(W))
+  int ntok;             // tokens per launch of the per-tile kernel (lq_decode_tokens)
 };
 
 constexpr uint32_t kWaitLimitDefault = 1u << 24;
@@ -84,6 +91,7 @@ inline StagingLayout staging_layout(size_t B, size_t Hk, size_t Hv, size_t d, si
 }
 
 cudaError_t launch_decode(const KParams &p, cudaStream_t stream);
+cudaError_t launch_decode_tokens(const KParams &p, cudaStream_t stream);
 cudaError_t launch_init(const KParams &p, cudaStream_t stream);
 cudaError_t launch_prefill(const KParams &p, cudaStream_t stream);
 cudaError_t launch_flush(const KParams &p, cudaStream_t stream);

@@ -27,7 +27,7 @@ def _declared():
 
 def test_exports_every_declared_symbol(B):
     names = _declared()
-    assert len(names) == 17
+    assert len(names) == 18
     assert sorted(B.EXPORTED) == names
     for n in names:
         assert hasattr(B._lib, n), n
@@ -56,7 +56,7 @@ def test_layout_matches_page_accounting(B):
 
 
 @pytest.mark.parametrize("field,value,status", [
-    ("d", 96, 2), ("d", 256, 2), ("window", 0, 2), ("window", 17, 2), ("n_comp", 9, 2),
+    ("d", 96, 2), ("d", 256, 2), ("window", 0, 2), ("window", 33, 2), ("n_comp", 9, 2),
     ("n_comp", -1, 2), ("smooth", 0.25, 2), ("batch", -1, 1), ("num_k_heads", 0, 1),
     ("num_v_heads", 3, 1), ("gate", 2, 1), ("in_dtype", 5, 1),
 ])

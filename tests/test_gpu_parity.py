@@ -96,6 +96,11 @@ CASES = {
     "naive_w1_k0": (wl.Workload("n", 1, 1, 2, 32, wl.GATE_SCALAR, False, 12, window=1,
                                 n_comp=0, smooth=0.0), 12),
     "gdn_d128_f32": (wl.Workload("gf", 2, 2, 4, 128, wl.GATE_SCALAR, False, 36), 36),
+    # windows above 16 tokens (the per-tile kernel): two folds of 32 tokens
+    "gdn_gva_d128_w32": (wl.Workload("g32", 2, 2, 4, 128, wl.GATE_SCALAR, True, 70,
+                                     window=32), 70),
+    "kda_d64_w32_k8": (wl.Workload("k32", 2, 2, 2, 64, wl.GATE_DIAG, False, 40, window=32,
+                                   n_comp=8), 40),
     "kda_d128_f32": (wl.Workload("kf", 2, 2, 2, 128, wl.GATE_DIAG, False, 36,
                                  v_outlier_channels=4), 36),
 }
@@ -225,6 +230,9 @@ RAGGED_CASES = {
     # KDA with bf16 inputs at d = 128 (the Kimi-Linear-like shape, fewer tiles)
     "kda_d128_bf16": wl.Workload("rk", 5, 8, 8, 128, wl.GATE_DIAG, True, 48,
                                  v_outlier_channels=4),
+    # a 32-token window: decode on the per-tile kernel, flushes of up to 31
+    # buffered tokens
+    "gdn_d64_bf16_w32": wl.Workload("r32", 5, 2, 4, 64, wl.GATE_SCALAR, True, 48, window=32),
 }
 
 
@@ -294,19 +302,21 @@ def test_active_mask_and_flush(case):
     assert B.lq_get_last_error(ds.st) == B.LQ_OK
 
 
-def test_dequantize_base_and_current_state():
-    w = wl.Workload("q", 2, 2, 2, 64, wl.GATE_DIAG, False, 21)
+@pytest.mark.parametrize("window,T", [(16, 21), (32, 45)])
+def test_dequantize_base_and_current_state(window, T):
+    w = wl.Workload("q", 2, 2, 2, 64, wl.GATE_DIAG, False, T, window=window)
     rng = np.random.default_rng(9)
     S0, _, _ = wl.initial_states(rng, w.tiles, w.d, w.d)
-    ti = wl.token_inputs(rng, w, 21)
+    ti = wl.token_inputs(rng, w, T)
     cfg = B.config_for(w)
     ds, tiles = _init_both(w, cfg, S0)
+    P.import_records(ds, [tl.rec for tl in tiles])     # one start record on both sides
     dev = P.DeviceInputs(ti, False)
     out = torch.empty((w.batch, w.num_v_heads, w.d), dtype=torch.float32, device="cuda")
-    for t in range(21):
+    for t in range(T):
         B.lq_decode_step(cfg, *dev.token(t), ds.st, out)
     for tl_i, tl in enumerate(tiles):
-        tl.run(*P.tile_inputs(ti, w, tl_i, 0, 21))
+        tl.run(*P.tile_inputs(ti, w, tl_i, 0, T))
     S_base = torch.empty((w.tiles, w.d, w.d), dtype=torch.float32, device="cuda")
     S_cur = torch.empty_like(S_base)
     B.lq_state_dequantize(cfg, ds.st, False, S_base)

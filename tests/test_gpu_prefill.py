@@ -1,4 +1,5 @@
-"""lq_prefill: the exact recurrence over a prompt, then the quantizer.
+"""lq_prefill: the exact recurrence over a prompt in chunks of 16 tokens (WY
+form, products with the state on the tf32 tensor path), then the quantizer.
 
 Outputs are compared with the oracle's exact fp64 recurrence, the record with
 the oracle's quantizer applied to the exact final state (codes within one
@@ -27,6 +28,10 @@ CASES = {
     "gdn_f32_d64_zero_start": (wl.Workload("p64", 2, 2, 4, 64, wl.GATE_SCALAR, False, 1),
                                80, False),
     "tiny_d32": (wl.Workload("p32", 1, 1, 2, 32, wl.GATE_SCALAR, False, 1), 50, True),
+    # a last chunk of one token, KDA at d = 32
+    "kda_f32_d32_T17": (wl.Workload("pk32", 2, 1, 2, 32, wl.GATE_DIAG, False, 1), 17, True),
+    # a prompt shorter than one chunk
+    "gdn_bf16_d128_T5": (wl.Workload("p5", 1, 2, 4, 128, wl.GATE_SCALAR, True, 1), 5, True),
 }
 
 

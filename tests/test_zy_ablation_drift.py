@@ -13,6 +13,10 @@ lowers the median drift against the configuration without it:
 - K = 4 compensator lines against none, both W = 16 with smoothing 1/2;
 - smoothing 1/2 against none, both W = 16 and K = 4.
 
+Longer windows keep lowering it: W = 32 (run on the per-tile kernel that
+serves windows above 16 tokens) must beat W = 16, and W = 16 must beat
+W = 8.
+
 The full LeapQuant configuration must also beat naive per-token int8.  The
 drift table is printed (pytest -s)."""
 import numpy as np
@@ -32,6 +36,7 @@ VARIANTS = [
     ("leapquant W16 K4 s1/2", 16, 4, 0.5),
     ("window W1 (K4 s1/2)", 1, 4, 0.5),
     ("window W8 (K4 s1/2)", 8, 4, 0.5),
+    ("window W32 (K4 s1/2)", 32, 4, 0.5),
     ("no compensators K0", 16, 0, 0.5),
     ("K2", 16, 2, 0.5),
     ("K8", 16, 8, 0.5),
@@ -99,6 +104,7 @@ def test_each_technique_lowers_drift_on_gpu():
               f"{drift.max():.2e}")
 
     full = med["leapquant W16 K4 s1/2"]
+    assert med["window W32 (K4 s1/2)"] < full < med["window W8 (K4 s1/2)"]
     assert full < med["window W1 (K4 s1/2)"]
     assert full < med["no compensators K0"]
     assert full < med["no smoothing s0"]
