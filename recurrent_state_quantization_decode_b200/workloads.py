@@ -151,3 +151,37 @@ def ragged_lengths(rng: np.random.Generator, n: int, mu: float = 7.0, sigma: flo
     L = np.clip(np.rint(rng.lognormal(mu, sigma, n)), 1, max_len).astype(np.int64)
     phase = rng.integers(0, 16, n).astype(np.int64)
     return L, phase
+
+
+def token_inputs_device(gen, w: Workload, T: int, device, batch: Optional[int] = None) -> dict:
+    """T tokens of inputs for workload w drawn on the device with a seeded
+    torch.Generator, by the same recipe as token_inputs (q, k ~ N(0, 1)
+    L2-normalised per head, v ~ N(0, 1), beta = sigmoid(N(0, 1)), GDN alpha ~
+    U(0.9, 1), KDA alpha = exp(-softplus(N(0, 1)) 0.05), q, k, v rounded to bf16
+    for bf16 workloads).  For batches too large to draw on the host every
+    token; returns torch tensors q, k [T, B, Hk, d], v [T, B, Hv, d] (bf16 or
+    fp32), alpha, beta fp32."""
+    import torch
+
+    B = w.batch if batch is None else batch
+    Hk, Hv, d = w.num_k_heads, w.num_v_heads, w.d
+
+    def normal(*shape):
+        return torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+
+    def unit(x):
+        return x / torch.linalg.vector_norm(x.double(), dim=-1, keepdim=True).clamp_min(1e-30).float()
+
+    q, k = unit(normal(T, B, Hk, d)), unit(normal(T, B, Hk, d))
+    v = normal(T, B, Hv, d)
+    if w.v_outlier_channels:
+        ch = np.random.default_rng(12345).choice(d, w.v_outlier_channels, replace=False)
+        v[..., torch.as_tensor(ch, device=device)] *= 10.0
+    beta = torch.sigmoid(normal(T, B, Hv))
+    if w.gate == GATE_SCALAR:
+        alpha = 0.9 + 0.1 * torch.rand((T, B, Hv), generator=gen, device=device)
+    else:
+        alpha = torch.exp(-torch.nn.functional.softplus(normal(T, B, Hv, d)) * 0.05)
+    dt = torch.bfloat16 if w.io_bf16 else torch.float32
+    return {"q": q.to(dt), "k": k.to(dt), "v": v.to(dt), "alpha": alpha.contiguous(),
+            "beta": beta.contiguous()}

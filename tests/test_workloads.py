@@ -105,3 +105,32 @@ def test_same_seed_same_inputs():
     b = wl.token_inputs(np.random.default_rng(7), w, 5)
     for n in ("q", "k", "v", "alpha", "beta"):
         np.testing.assert_array_equal(getattr(a, n), getattr(b, n))
+
+
+def test_device_generator_follows_the_recipe():
+    """token_inputs_device (the draws for batches too large for the host) keeps
+    the recipe of token_inputs: unit-norm q and k per head (bf16-rounded),
+    beta in (0, 1), GDN alpha in [0.9, 1], KDA alpha in (0, 1], shapes, and
+    the same stream for the same seed (checked on the CPU device)."""
+    import torch
+
+    for w in (wl.RAGGED, wl.KIMI_LINEAR_KDA):
+        g1, g2 = torch.Generator(), torch.Generator()
+        g1.manual_seed(3)
+        g2.manual_seed(3)
+        a = wl.token_inputs_device(g1, w, 3, "cpu", batch=2)
+        b = wl.token_inputs_device(g2, w, 3, "cpu", batch=2)
+        for n in a:
+            assert torch.equal(a[n], b[n]), n
+        assert a["q"].shape == (3, 2, w.num_k_heads, w.d)
+        assert a["v"].shape == (3, 2, w.num_v_heads, w.d)
+        assert a["q"].dtype == torch.bfloat16 and a["v"].dtype == torch.bfloat16
+        nq = torch.linalg.vector_norm(a["q"].double(), dim=-1)
+        assert torch.allclose(nq, torch.ones_like(nq), atol=1e-2)
+        assert torch.all((a["beta"] > 0) & (a["beta"] < 1))
+        if w.gate == wl.GATE_SCALAR:
+            assert a["alpha"].shape == (3, 2, w.num_v_heads)
+            assert torch.all((a["alpha"] >= 0.9) & (a["alpha"] <= 1.0))
+        else:
+            assert a["alpha"].shape == (3, 2, w.num_v_heads, w.d)
+            assert torch.all((a["alpha"] > 0) & (a["alpha"] <= 1.0))

@@ -1,6 +1,10 @@
-"""Long ragged continuous batch: the long-decode workload (ragged lengths
-~ LogNormal(7, 1), per-sequence window phases, a checkpoint every 1,024
-tokens) at a reduced size, through the C-ABI decode step.
+"""Long ragged continuous batch: the long-decode workload at its stated size
+(256 sequences x 32 heads, GDN, d = 128, ragged lengths ~ LogNormal(7, 1),
+per-sequence window phases, a checkpoint every 1,024 tokens), through the
+C-ABI decode step.  The sampled tiles' inputs are drawn on the host (numpy,
+seeded) and also feed the oracle; every other tile's inputs are drawn on the
+device by the same recipe (torch, seeded), since the whole batch is too
+large to draw on the host token by token.
 
 It checks three things:
 
@@ -30,7 +34,7 @@ from recurrent_state_quantization_decode_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
 
-B_SEQ, HK, HV, D = 16, 16, 32, 128
+B_SEQ, HK, HV, D = wl.RAGGED.batch, wl.RAGGED.num_k_heads, wl.RAGGED.num_v_heads, wl.RAGGED.d
 CHUNK = 128                      # tokens drawn per host batch
 CKPT = 1024                      # checkpoint cadence in absolute positions
 MAX_LEN = int(os.environ.get("LQ_LONG_DECODE_MAX_LEN", "4096"))
@@ -95,16 +99,25 @@ def test_long_ragged_decode_checkpoint_resume_and_drift():
     slots = torch.full((B_SEQ,), -1, dtype=torch.int32, device="cuda")
     slots[rb] = 0
     dev_chunks = []
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(11)
+    smp_w = wl.Workload("ragged_sampled", len(sample), 1, 1, D, wl.GATE_SCALAR, True, T)
+    smp_b_dev = torch.from_numpy(smp_b).cuda()
+    smp_h_dev = torch.from_numpy(smp_h).cuda()
+    smp_hk_dev = torch.from_numpy(smp_hk).cuda()
     for c0 in range(0, T, CHUNK):
-        ti = wl.token_inputs(rng, w, min(CHUNK, T - c0))
-        host_inputs["q"].append(ti.q[:, smp_b, smp_hk])
-        host_inputs["k"].append(ti.k[:, smp_b, smp_hk])
-        for n in ("v", "alpha", "beta"):
-            host_inputs[n].append(getattr(ti, n)[:, smp_b, smp_h])
-        dev = {n: torch.from_numpy(getattr(ti, n)).cuda() for n in ("q", "k", "v", "alpha",
-                                                                   "beta")}
-        for n in ("q", "k", "v"):
-            dev[n] = dev[n].to(torch.bfloat16)
+        n_tok = min(CHUNK, T - c0)
+        dev = wl.token_inputs_device(gen, w, n_tok, "cuda")
+        # the sampled tiles: host draws, written into the device inputs
+        ti = wl.token_inputs(rng, smp_w, n_tok)            # [n_tok, sample, 1, D]
+        host = {n: getattr(ti, n)[:, :, 0] for n in ("q", "k", "v", "alpha", "beta")}
+        for n in host:
+            host_inputs[n].append(host[n])
+        dev["q"][:, smp_b_dev, smp_hk_dev] = torch.from_numpy(host["q"]).cuda().to(torch.bfloat16)
+        dev["k"][:, smp_b_dev, smp_hk_dev] = torch.from_numpy(host["k"]).cuda().to(torch.bfloat16)
+        dev["v"][:, smp_b_dev, smp_h_dev] = torch.from_numpy(host["v"]).cuda().to(torch.bfloat16)
+        dev["alpha"][:, smp_b_dev, smp_h_dev] = torch.from_numpy(host["alpha"]).cuda()
+        dev["beta"][:, smp_b_dev, smp_h_dev] = torch.from_numpy(host["beta"]).cuda()
         dev_chunks.append(dev)
         for tt in range(dev["q"].shape[0]):
             t = c0 + tt
