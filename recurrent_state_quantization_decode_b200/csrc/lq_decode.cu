@@ -1188,11 +1188,14 @@ __device__ __forceinline__ void channel_chunk_fast(const KParams &p, TK &x,
 // digit scales, combines, reductions) are spread over four warps instead of
 // eight, and no CTA-wide barrier is taken on a plain token.
 
-// Sums 32 per-lane values over the warp: afterwards lane l holds the total of
-// value l (31 shuffles).
-__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
+// Sums NV (32 or 16) per-lane values over the warp: afterwards lane l holds
+// the total of value l * NV / 32 (NV - 1 shuffles, and one more for NV = 16).
+template <int NV>
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[NV], int lane) {
+  static_assert(NV == 32 || NV == 16, "32 or 16 values");
+  int step = 16;
 #pragma unroll
-  for (int step = 16, half = 16; step >= 1; step >>= 1, half >>= 1) {
+  for (int half = NV / 2; half >= 1; step >>= 1, half >>= 1) {
     const bool upper = (lane & step) != 0;
 #pragma unroll
     for (int i = 0; i < half; ++i) {
@@ -1201,6 +1204,7 @@ __device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) 
       v[i] = keep + __shfl_xor_sync(kFull, send, step);
     }
   }
+  if (NV == 16) v[0] += __shfl_xor_sync(kFull, v[0], 1);
   return v[0];
 }
 
@@ -1251,23 +1255,44 @@ __device__ __forceinline__ void quad_channel(const KParams &p, QTok<D> &x, const
   float G;
   if constexpr (KDA) {
     const float *sa = reinterpret_cast<const float *>(slot + lay.a);
-    // v[s]: this lane's share of c_s; v[16 + s]: of a_s (a_n = k . q)
-    float v[32];
+    // This lane's share of c_s (s < n) and a_s (s <= n, a_n = k . q), summed
+    // over the chunk by one transposed reduction: of 16 values while n < 8
+    // (c_0..7, a_0..7), of 32 otherwise.
     float rho = sa[j];
+    if (n < 8) {
+      float v[16];
 #pragma unroll
-    for (int s2 = kMaxWindow - 1; s2 >= 0; --s2) {
-      if (s2 < n) {
-        const float kr = __bfloat162float(sbk[s2 * D + j]) * rho;
-        v[s2] = kr * k;
-        v[16 + s2] = kr * q;
-        rho *= sbg[s2 * D + j];
-      } else {
-        v[s2] = 0.0f;
-        v[16 + s2] = (s2 == n) ? k * q : 0.0f;
+      for (int s2 = 7; s2 >= 0; --s2) {
+        if (s2 < n) {
+          const float kr = __bfloat162float(sbk[s2 * D + j]) * rho;
+          v[s2] = kr * k;
+          v[8 + s2] = kr * q;
+          rho *= sbg[s2 * D + j];
+        } else {
+          v[s2] = 0.0f;
+          v[8 + s2] = (s2 == n) ? k * q : 0.0f;
+        }
       }
+      const float tot = warp_transpose_sum<16>(v, lane);
+      const int vi = lane >> 1;
+      if ((lane & 1) == 0) x.cpk[w][vi < 8 ? vi : 8 + vi] = tot;
+    } else {
+      float v[32];
+#pragma unroll
+      for (int s2 = kMaxWindow - 1; s2 >= 0; --s2) {
+        if (s2 < n) {
+          const float kr = __bfloat162float(sbk[s2 * D + j]) * rho;
+          v[s2] = kr * k;
+          v[16 + s2] = kr * q;
+          rho *= sbg[s2 * D + j];
+        } else {
+          v[s2] = 0.0f;
+          v[16 + s2] = (s2 == n) ? k * q : 0.0f;
+        }
+      }
+      x.cpk[w][lane] = warp_transpose_sum<32>(v, lane);
     }
     G = rho;
-    x.cpk[w][lane] = warp_transpose_sum32(v, lane);
   } else {
     G = gate_product(sbg, alpha0, n);
     if (w == 0)
