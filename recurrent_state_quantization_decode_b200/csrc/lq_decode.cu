@@ -1479,28 +1479,29 @@ template <int D, bool KDA, class Src>
 __device__ __forceinline__ void quad_rows(const KParams &p, const QTok<D> &x, const Src &r,
                                           int tile, int n, float beta, int w) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  // the coefficients of this lane's buffer slots s = t + 4u
-  float cs[4], as[4];
+  // the coefficients of this lane's buffer slots s = t + 4u; KDA: lane l sums
+  // the four warps' partials of value l (c_l for l < 16, a_(l-16) above) once,
+  // and the lanes that need a value take it by shuffle
+  float cs[4], as[4], ann;
+  if constexpr (KDA) {
+    const float tot = (x.cpk[0][lane] + x.cpk[1][lane]) + (x.cpk[2][lane] + x.cpk[3][lane]);
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int s2 = t + 4 * u;
-    cs[u] = 0.0f;
-    as[u] = 0.0f;
-    if (s2 < n) {
-      if constexpr (KDA) {
-        cs[u] = (x.cpk[0][s2] + x.cpk[1][s2]) + (x.cpk[2][s2] + x.cpk[3][s2]);
-        as[u] = (x.cpk[0][16 + s2] + x.cpk[1][16 + s2]) + (x.cpk[2][16 + s2] + x.cpk[3][16 + s2]);
-      } else {
-        cs[u] = x.cc[s2];
-        as[u] = x.aa[s2];
-      }
+    for (int u = 0; u < 4; ++u) {
+      const int s2 = t + 4 * u;
+      const float c = __shfl_sync(kFull, tot, s2), a = __shfl_sync(kFull, tot, 16 + s2);
+      cs[u] = s2 < n ? c : 0.0f;
+      as[u] = s2 < n ? a : 0.0f;
     }
-  }
-  float ann;
-  if constexpr (KDA)
-    ann = (x.cpk[0][16 + n] + x.cpk[1][16 + n]) + (x.cpk[2][16 + n] + x.cpk[3][16 + n]);
-  else
+    ann = __shfl_sync(kFull, tot, 16 + n);
+  } else {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int s2 = t + 4 * u;
+      cs[u] = s2 < n ? x.cc[s2] : 0.0f;
+      as[u] = s2 < n ? x.aa[s2] : 0.0f;
+    }
     ann = x.aa[n];
+  }
   // this lane's compensator lines: column lines scale their values at the rows
   // by Gamma_j x_j; a row line adds its dots to the one row it is
   float cq[2], ck[2], rq[2], rk[2];
@@ -1996,23 +1997,24 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
     }
     fence_mbar_init();
   }
+  // The quad path's first records are fetched into L2 before the wait below:
+  // a prefetch consumes nothing, and L2 is where the previous kernel's writes
+  // land, so it cannot make a later copy read stale data.
+  if (kQuad && tid == 0)
+    for (int st = 0; st < kStages && st < mine; ++st)
+      prefetch_l2(p.records + static_cast<size_t>(blockIdx.x + st * gridDim.x) * p.L.bytes,
+                  static_cast<uint32_t>(p.L.bytes));
   // Launched as a programmatic dependent: everything above touched only this
-  // CTA's shared memory.  Wait here until the previous kernel in the stream
-  // has completed and its writes are visible, and let the next one start
-  // its own setup as this grid's CTAs retire.
+  // CTA's shared memory (and L2).  Wait here until the previous kernel in the
+  // stream has completed and its writes are visible, and let the next one
+  // start its own setup as this grid's CTAs retire.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (tid == 0) {
-    for (int st = 0; st < kStages && st < mine; ++st) {
-      const int tl = blockIdx.x + st * gridDim.x;
-      if (speculate) {
-        if (!(p.withhold && blockIdx.x == 0 && st == 0))
-          issue_record<D, BF16, KDA>(p, smem + st * slot_bytes, &s.bar[st], tl);
-      } else if (kQuad) {
-        prefetch_l2(p.records + static_cast<size_t>(tl) * p.L.bytes,
-                    static_cast<uint32_t>(p.L.bytes));
-      }
-    }
+  if (speculate && tid == 0) {
+    for (int st = 0; st < kStages && st < mine; ++st)
+      if (!(p.withhold && blockIdx.x == 0 && st == 0))
+        issue_record<D, BF16, KDA>(p, smem + st * slot_bytes, &s.bar[st],
+                                   blockIdx.x + st * gridDim.x);
   }
   int keep = 0, tile = 0, n = -1, coord = 0;
   float a0 = 0.0f, b0 = 0.0f;
