@@ -982,6 +982,11 @@ __device__ __forceinline__ void issue_rest(const KParams &p, uint8_t *slot,
   if (KDA) bulk_g2s(slot + lay.a, p.alpha + static_cast<size_t>(tile) * D, D * 4, bar);
 }
 
+// L2 prefetch of `bytes` at `src` (16-byte aligned, a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // GDN with bf16 inputs: the buffer coefficients of all slots from one warp.
 // Raw dots k_s . k_t and k_s . q_t for slots s = 0..15 run on the bf16 tensor
 // path (keys and queries are bf16, so every product is exact; fp32
@@ -1294,7 +1299,13 @@ __device__ __forceinline__ void quad_channel(const KParams &p, QTok<D> &x, const
     }
     G = rho;
   } else {
-    G = gate_product(sbg, alpha0, n);
+    // Gamma = the product of the n buffered gates and the current one: lane s
+    // holds gate s (1 past n), multiplied over the warp by a butterfly whose
+    // pairs are the same in every lane, so every lane gets the same bits
+    float a = lane < n ? sbg[lane] : (lane == n ? alpha0 : 1.0f);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a *= __shfl_xor_sync(kFull, a, o);
+    G = a;
     if (w == 0)
       coef_mma<D>(x, sbk, sk, sq, sbg, alpha0, n);
   }
@@ -1960,10 +1971,6 @@ __device__ __forceinline__ bool wait_issued(const int *slot_last, int e, uint32_
   return false;
 }
 
-// L2 prefetch of `bytes` at `src` (16-byte aligned, a multiple of 16).
-__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 
 template <int D, bool BF16, bool KDA>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
@@ -2106,6 +2113,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const KParams p) {
       uint8_t *slot = smem + st * slot_bytes;
       QTok<D> &x = s.u.qt[quad][li & 1];
       const int tl = s.tl_tile[e], ne = s.tl_n[e];
+
       quad_channel<D, KDA>(p, x, slot, tl, ne, s.tl_coord[e], s.tl_a[e], w, ok);
       if constexpr (TR::kEarlyRelease) {
         // everything the rows need from the slot goes to registers now, so
