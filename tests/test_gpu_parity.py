@@ -101,6 +101,13 @@ CASES = {
                                      window=32), 70),
     "kda_d64_w32_k8": (wl.Workload("k32", 2, 2, 2, 64, wl.GATE_DIAG, False, 40, window=32,
                                    n_comp=8), 40),
+    # the quad path (d = 128, bf16 inputs) without compensators, with eight of
+    # them (larger records, fewer CTAs per SM), and with smoothing off / full
+    "gdn_gva_d128_k0": (wl.Workload("gk0", 2, 4, 8, 128, wl.GATE_SCALAR, True, 20, n_comp=0), 20),
+    "kda_d128_k8_s1": (wl.Workload("kk8", 2, 4, 4, 128, wl.GATE_DIAG, True, 20, n_comp=8,
+                                   smooth=1.0), 20),
+    "gdn_gva_d128_s0": (wl.Workload("gs0", 2, 4, 8, 128, wl.GATE_SCALAR, True, 20,
+                                    smooth=0.0), 20),
     "kda_d128_f32": (wl.Workload("kf", 2, 2, 2, 128, wl.GATE_DIAG, False, 36,
                                  v_outlier_channels=4), 36),
 }
@@ -170,8 +177,10 @@ def test_decode_free_running_tiny_workload():
     P.assert_records_close(diff)
 
 
-def test_bf16_output():
-    w = wl.Workload("g", 2, 2, 4, 64, wl.GATE_SCALAR, True, 20)
+@pytest.mark.parametrize("d,gate", [(64, wl.GATE_SCALAR), (128, wl.GATE_SCALAR),
+                                    (128, wl.GATE_DIAG)])
+def test_bf16_output(d, gate):
+    w = wl.Workload("g", 2, 2, 4, d, gate, True, 20)
     rng = np.random.default_rng(3)
     S0, _, _ = wl.initial_states(rng, w.tiles, w.d, w.d)
     ti = wl.token_inputs(rng, w, 20)
