@@ -399,10 +399,24 @@ class Layer:
             torch.cuda.synchronize(device)
 
     def pin_host_inputs(self):
+        """Pinned host copies of the W tokens' inputs: per token, q, k, v,
+        alpha and beta back to back in one block, which lq_decode_step_host
+        moves with one copy."""
         import torch
 
-        self.host = {n: getattr(self, n).cpu().pin_memory()
-                     for n in ("q", "k", "v", "alpha", "beta")}
+        names = ("q", "k", "v", "alpha", "beta")
+        W = self.q.shape[0]
+        sizes = [getattr(self, n)[0].numel() * getattr(self, n)[0].element_size() for n in names]
+        block = torch.empty((W, sum(sizes)), dtype=torch.uint8).pin_memory()
+        self.host = {n: [] for n in names}
+        for t in range(W):
+            off = 0
+            for n, sz in zip(names, sizes):
+                x = getattr(self, n)[t].cpu()
+                view = block[t, off:off + sz].view(x.dtype).view(x.shape)
+                view.copy_(x)
+                self.host[n].append(view)
+                off += sz
         self.host_out = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
         self.staging = torch.empty(self.ds.layout.host_staging_bytes, dtype=torch.uint8,
                                    device=self.out.device)
@@ -724,9 +738,9 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
         ms_e2e = max_over_ranks(start.elapsed_time(end), world, device)
         e2e = {"value": whole_job_rate(units_per_step, world, e2e_steps, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "path": ("lq_decode_step_host: pinned host q, k, v, alpha, beta read over "
-                        "the host link by the gather kernel, o back by cudaMemcpyAsync; "
-                        f"{len(streams)} streams by layer index")}
+               "path": ("lq_decode_step_host: each token's pinned host q, k, v, alpha, "
+                        "beta back to back, moved by one cudaMemcpyAsync, o back by "
+                        f"cudaMemcpyAsync; {len(streams)} streams by layer index")}
 
     # prefill of one layer's tiles over a prompt, ending in the quantizer
     prefill = None

@@ -220,7 +220,13 @@ lq_status lq_decode_tokens(const lq_config *cfg, int32_t ntok, const void *q, co
  * (the call reads out_host's current rows into the staging before the step and
  * copies the whole output region back), so out_host must stay unchanged by
  * the host until the stream reaches the output copy.
- *  - Inputs in pinned memory that the device maps at the same address
+ *  - Inputs that sit back to back in host memory in the order q, k, v,
+ *    alpha, beta, when each of their sizes is a multiple of 256 bytes (so
+ *    that the staging holds them back to back too), are moved by one
+ *    cudaMemcpyAsync: a single copy-engine start-up, and no SM held while
+ *    the bytes cross the host link, so that the copy overlaps kernels of
+ *    other streams.
+ *  - Otherwise, inputs in pinned memory that the device maps at the same address
  *    (cudaHostAlloc / cudaMallocHost memory under unified addressing, as the
  *    driver reports through cudaPointerGetAttributes for both ends of the
  *    input) are read by one gather kernel over the host link: a token's small

@@ -343,8 +343,24 @@ lq_status lq_decode_step_host(const lq_config *cfg, const void *q_host, const vo
   const size_t bytes[6] = {sl.q_bytes, sl.q_bytes, sl.v_bytes, sl.alpha_bytes, sl.beta_bytes,
                            sl.out_bytes};
   const int nsrc = active != nullptr ? 6 : 5;
+  // Inputs back to back in host memory, in the staging's order and with its
+  // spacing (every input a multiple of 256 bytes, so that the staging has no
+  // gaps): one copy-engine copy moves them all and occupies no SM, so that it
+  // overlaps kernels of other streams.
+  bool packed = true;
+  for (int i = 1; i < 5; ++i)
+    packed = packed && dst[i] == static_cast<uint8_t *>(dst[i - 1]) + bytes[i - 1] &&
+             src[i] == static_cast<const uint8_t *>(src[i - 1]) + bytes[i - 1];
+  int first = 0;
+  if (packed) {
+    const size_t span = static_cast<size_t>(static_cast<uint8_t *>(dst[4]) + bytes[4] -
+                                            static_cast<uint8_t *>(dst[0]));
+    if (cudaMemcpyAsync(dst[0], src[0], span, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+      return LQ_ERR_CUDA;
+    first = 5;
+  }
   lq::GatherList gather{};
-  for (int i = 0; i < nsrc; ++i) {
+  for (int i = first; i < nsrc; ++i) {
     if (const void *view = lq::device_view_of_host(src[i], bytes[i])) {
       gather.seg[gather.n++] = lq::GatherSeg{view, dst[i], bytes[i]};
     } else if (cudaMemcpyAsync(dst[i], src[i], bytes[i], cudaMemcpyHostToDevice, cs) !=

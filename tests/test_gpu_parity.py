@@ -488,7 +488,30 @@ HOST_MODES = {
     # a 16-byte boundary in pinned memory (the bytewise path)
     "ragged_misaligned": (wl.Workload("h9", 3, 1, 3, 64, wl.GATE_SCALAR, True, 20),
                           set("qkv") | {"alpha", "beta"}),
+    # each token's q, k, v, alpha, beta back to back in one pinned block (every
+    # size a multiple of 256 bytes): one copy-engine copy per call; GDN and KDA
+    "packed": (wl.Workload("hp", 16, 2, 4, 128, wl.GATE_SCALAR, True, 20), set()),
+    "packed_kda": (wl.Workload("hpk", 16, 4, 4, 128, wl.GATE_DIAG, True, 20), set()),
 }
+
+
+def _packed_host_inputs(dev, T):
+    """Per token, q, k, v, alpha, beta back to back in one pinned block."""
+    names = ("q", "k", "v", "alpha", "beta")
+    sizes = [getattr(dev, n)[0].numel() * getattr(dev, n)[0].element_size() for n in names]
+    assert all(sz % 256 == 0 for sz in sizes)
+    block = torch.empty((T, sum(sizes)), dtype=torch.uint8).pin_memory()
+    host = {n: [] for n in names}
+    for t in range(T):
+        off = 0
+        for n, sz in zip(names, sizes):
+            x = getattr(dev, n)[t].cpu()
+            view = block[t, off:off + sz].view(x.dtype).view(x.shape)
+            view.copy_(x)
+            host[n].append(view)
+            off += sz
+        assert host["k"][t].data_ptr() == host["q"][t].data_ptr() + sizes[0]
+    return host
 
 
 @pytest.mark.parametrize("mode", sorted(HOST_MODES))
@@ -504,8 +527,8 @@ def test_host_entry_point_matches_device_entry_point(mode):
     B.lq_state_init(cfg, S0_dev, a.st)
     B.lq_state_init(cfg, S0_dev, b.st)
     dev = P.DeviceInputs(ti, True)
-    host = {}
-    for n in ("q", "k", "v", "alpha", "beta"):
+    host = _packed_host_inputs(dev, 20) if mode.startswith("packed") else {}
+    for n in ("q", "k", "v", "alpha", "beta") if not host else ():
         x = getattr(dev, n).cpu()
         if n in pinned and mode == "ragged_misaligned" and n in ("alpha", "beta"):
             buf = torch.empty(x.numel() + 1, dtype=x.dtype).pin_memory()
