@@ -700,11 +700,11 @@ def gpu_arm(args, w: wl.Workload, rank: int, world: int, local_rank: int) -> Non
         d2h = sum(ly.host_out.numel() * 4 for ly in layers) * W
         e2e_steps = max(2, min(args.steps, 20))
 
-        # Four streams, layer index mod 4 picks one (fewer when L is not a
+        # Eight streams, layer index mod 8 picks one (fewer when L is not a
         # multiple): each layer stays on its own stream (its tokens in order,
-        # its own staging and output buffers), while one layer's input gather
+        # its own staging and output buffers), while one layer's input copy
         # and output copy overlap other layers' kernels.
-        n_streams = 4 if L % 4 == 0 else (2 if L % 2 == 0 else 1)
+        n_streams = next(n for n in (8, 4, 2, 1) if L % n == 0)
         streams = [stream] + [torch.cuda.Stream(device=device) for _ in range(n_streams - 1)]
 
         def step_host():
