@@ -117,10 +117,17 @@ def fp32_bytes_per_tile_step(w: wl.Workload, out_bytes: int = 4) -> float:
     return 2 * 4 * d * d + 2 * inb * d / g + inb * d + 4 * ga + 4 + out_bytes * d
 
 
+_COMMENTS = re.compile(rb"/\*.*?\*/|//[^\n]*", re.S)
+
+
 def kernel_source_sha() -> str:
+    """Hash of the decode kernel's source with its comments left out and its
+    whitespace collapsed, so that a change of wording or layout alone keeps a
+    profile summary tied to the kernel that it measured."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        h.update(open(f, "rb").read())
+        code = _COMMENTS.sub(b" ", open(f, "rb").read())
+        h.update(re.sub(rb"\s+", b" ", code).strip())
     return h.hexdigest()[:16]
 
 

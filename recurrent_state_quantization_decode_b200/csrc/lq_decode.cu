@@ -27,15 +27,21 @@
 //    product up to the digits' truncation (<= 7.5e-9 max|x| per element) and
 //    one rounding per combination step.  No code is ever converted to float on
 //    this path.
-//  * GDN with bf16 inputs takes a shorter per-token path with one CTA barrier
-//    per tile.  Each int8 k-chunk (32 key channels) has its own digit scale,
-//    so one warp per chunk does that chunk's per-channel work (gate product, x,
-//    its max, digits, compensator dots) without a CTA-wide max; one warp gets
-//    the buffer coefficients c_s = rho_s k_s . k and a_s = rho_s k_s . q from a
-//    bf16 m16n8k16 product; the other row warps fetch their codes meanwhile.
-//    The per-token values are double-buffered, so a warp may start the next
-//    tile while others finish the current one, and every thread waits on the
-//    slot's mbarrier itself.
+//  * Plain tokens of d = 128 tiles with bf16 inputs (GDN and KDA) run on the
+//    quad path: four warps take one tile and a CTA runs two tiles at once.
+//    Warp w of a quad does the per-channel work of int8 k-chunk w (32 key
+//    channels, its own digit scale: gate product or KDA decay ratios and the
+//    chunk's share of the buffer coefficients, x, digits, compensator dots),
+//    then, after the quad's one named barrier, finishes state rows 32w ..
+//    32w + 31.  Boundary tokens, the list's last entries, run on the whole CTA.
+//  * On the whole-CTA path (every token at d < 128, boundary tokens at
+//    d = 128) GDN with bf16 inputs has one CTA barrier per tile before the
+//    fold: one warp per k-chunk for the per-channel work, one warp for the
+//    buffer coefficients c_s = rho_s k_s . k and a_s = rho_s k_s . q from a
+//    bf16 m16n8k16 product, the other row warps fetching their codes
+//    meanwhile.  The per-token values are double-buffered, so a warp may start
+//    the next tile while others finish the current one, and every thread waits
+//    on the slot's mbarrier itself.
 //  * On the boundary token the fp32 state S = S0 diag(Gamma) + sum d_s kt_s^T
 //    is built in registers, in the same fragment layout as the codes: the
 //    dequantized base, then (d >= 64) the rank-W update on the tf32 tensor

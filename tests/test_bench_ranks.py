@@ -161,7 +161,7 @@ def test_algorithmic_bytes_and_profiled_traffic(tmp_path, monkeypatch):
     assert bench.fp32_bytes_per_tile_step(w) == 2 * 4 * d * d + 520 + 4 * d
 
     src = tmp_path / "kernel.cu"
-    src.write_text("// kernel v1\n")
+    src.write_text("// kernel\nint v = 1;\n")
     monkeypatch.setattr(bench, "KERNEL_SOURCES", [str(src)])
     summary = tmp_path / "decode_kernel_qwen35_9b_gdn.md"
     monkeypatch.setattr(bench, "PROFILE_DIR", str(tmp_path))
@@ -171,7 +171,9 @@ def test_algorithmic_bytes_and_profiled_traffic(tmp_path, monkeypatch):
                        "dram_bytes_per_tile_step: 24911\n")
     assert bench.profiled_traffic(2048) == 24911 * 2048
     assert bench.profiled_traffic(4096, "kimi_linear_kda") is None   # another workload's file
-    src.write_text("// kernel v2\n")                            # kernel changed since
+    src.write_text("/* the kernel,\n   reworded */ int v = 1;  // same code\n")
+    assert bench.profiled_traffic(2048) == 24911 * 2048        # comments alone changed
+    src.write_text("// kernel\nint v = 2;\n")                  # kernel changed since
     assert bench.profiled_traffic(2048) is None
     # the roofline names the kernel instance of each workload
     assert bench.kernel_label(bench.WORKLOADS["kimi_linear_kda"]).startswith(
