@@ -396,6 +396,15 @@ class Layer:
         self.alpha = torch.from_numpy(ti.alpha).to(device)
         self.beta = torch.from_numpy(ti.beta).to(device)
         self.out = torch.empty((w.batch, w.num_v_heads, w.d), dtype=torch.float32, device=device)
+        # Without grouped heads (Hv = Hk) each token's inputs are also kept in
+        # lq_decode_step_packed's per-tile blocks, which the int8 step reads
+        # (one copy per tile instead of four); with grouped heads the blocks
+        # would repeat q and k per value head, so those layers keep the
+        # separate arrays.
+        self.packed = None
+        if w.num_v_heads == w.num_k_heads:
+            self.packed = [B.pack_tile_inputs(self.cfg, self.q[t], self.k[t], self.v[t],
+                                              self.alpha[t]) for t in range(w.window)]
         self.host = None
         if phases is not None:
             ph = torch.as_tensor(phases, dtype=torch.int32, device=device)
@@ -560,8 +569,13 @@ def measure_decode(B, w: wl.Workload, key: str, L: int, steps: int, warmup: int,
     def step_int8(s):
         for t in range(W):
             for ly in layers:
-                B.lq_decode_step(ly.cfg, ly.q[t], ly.k[t], ly.v[t], ly.alpha[t], ly.beta[t],
-                                 ly.ds.st, ly.out, stream=s)
+                if ly.packed is not None:
+                    kda = ly.cfg.gate == B.LQ_GATE_DIAG
+                    B.lq_decode_step_packed(ly.cfg, ly.packed[t], None if kda else ly.alpha[t],
+                                            ly.beta[t], ly.ds.st, ly.out, stream=s)
+                else:
+                    B.lq_decode_step(ly.cfg, ly.q[t], ly.k[t], ly.v[t], ly.alpha[t], ly.beta[t],
+                                     ly.ds.st, ly.out, stream=s)
 
     def step_fp32(s):
         for t in range(W):

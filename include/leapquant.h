@@ -211,6 +211,23 @@ lq_status lq_decode_tokens(const lq_config *cfg, int32_t ntok, const void *q, co
                            const void *v, const float *alpha, const float *beta,
                            const lq_state *st, void *out, const int32_t *active, void *stream);
 
+/* lq_decode_step with the token's inputs packed per tile: the same step, the
+ * same results.  qkva: [B][Hv] blocks back to back, 16-byte aligned, one per
+ * tile (sequence b, value head h): q and k of key head h / (Hv / Hk), v of the
+ * tile (d values each, in_dtype), then for KDA the tile's gate alpha (d
+ * fp32).  A block is 3 d sizeof(in_dtype) (+ 4 d for KDA) bytes.  For GDN,
+ * alpha stays a separate [B][Hv] fp32 array; for KDA alpha must be NULL or is
+ * ignored.  beta, out and active as for lq_decode_step.
+ *  - Why: each of a tile's inputs is otherwise a bulk copy of its own into
+ *    shared memory, and four small copies per tile cost more than their
+ *    bytes; a block comes in one.  With grouped heads (Hv > Hk) the caller
+ *    writes q and k once per value head.
+ *  - W up to 16 only (LQ_ERR_UNSUPPORTED above); arguments are checked as for
+ *    lq_decode_step (qkva 16-byte aligned). */
+lq_status lq_decode_step_packed(const lq_config *cfg, const void *qkva, const float *alpha,
+                                const float *beta, const lq_state *st, void *out,
+                                const int32_t *active, void *stream);
+
 /* lq_decode_step with the token's inputs and output in HOST memory: moves
  * q, k, v, alpha, beta to `staging` (device, layout.host_staging_bytes,
  * 16-byte aligned), runs the step, and copies o back to out_host, all

@@ -35,7 +35,8 @@ EXPORTED = ("lq_version", "lq_status_string", "lq_state_layout", "lq_state_bytes
             "lq_decode_step_host_noalloc", "lq_window_flush",
             "lq_fp32_decode_step", "lq_state_dequantize", "lq_get_last_error",
             "lq_test_decode_step_timeout", "lq_prefill", "lq_checkpoint_save",
-            "lq_checkpoint_restore", "lq_window_rewind", "lq_decode_tokens")
+            "lq_checkpoint_restore", "lq_window_rewind", "lq_decode_tokens",
+            "lq_decode_step_packed")
 
 
 class lq_config(ctypes.Structure):
@@ -70,6 +71,7 @@ _sig = {
                         ctypes.POINTER(ctypes.c_size_t)], ctypes.c_size_t),
     "lq_state_init": ([_CFG, _P, _ST, _P, _P], ctypes.c_int),
     "lq_decode_step": ([_CFG, _P, _P, _P, _P, _P, _ST, _P, _P, _P], ctypes.c_int),
+    "lq_decode_step_packed": ([_CFG, _P, _P, _P, _ST, _P, _P, _P], ctypes.c_int),
     "lq_decode_step_host": ([_CFG, _P, _P, _P, _P, _P, _ST, _P, _P, _P, _P], ctypes.c_int),
     "lq_decode_step_host_noalloc": ([_CFG, _P, _P, _P, _P, _P, _ST, _P, _P, _P], ctypes.c_int),
     "lq_window_flush": ([_CFG, _ST, _P, _P], ctypes.c_int),
@@ -180,6 +182,30 @@ def lq_decode_step(cfg, q, k, v, alpha, beta, state: lq_state, out, active=None,
     _check(_lib.lq_decode_step(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
                                _ptr(beta), ctypes.byref(state), _ptr(out), _ptr(active),
                                _stream(stream)), "lq_decode_step")
+
+
+def lq_decode_step_packed(cfg, qkva, alpha, beta, state: lq_state, out, active=None,
+                          stream=None) -> None:
+    """lq_decode_step with each tile's q, k, v (and KDA gate) packed back to
+    back in qkva (see pack_tile_inputs); alpha: the GDN gates, None for KDA."""
+    _check(_lib.lq_decode_step_packed(ctypes.byref(cfg), _ptr(qkva), _ptr(alpha), _ptr(beta),
+                                      ctypes.byref(state), _ptr(out), _ptr(active),
+                                      _stream(stream)), "lq_decode_step_packed")
+
+
+def pack_tile_inputs(cfg, q, k, v, alpha):
+    """The per-tile block layout of lq_decode_step_packed from q, k [B][Hk][d],
+    v [B][Hv][d] and, for KDA, alpha [B][Hv][d] (torch tensors on one device):
+    a uint8 tensor [B][Hv][block bytes]."""
+    import torch
+
+    B, Hk, Hv = cfg.batch, cfg.num_k_heads, cfg.num_v_heads
+    g = Hv // Hk
+    parts = [q.repeat_interleave(g, dim=1), k.repeat_interleave(g, dim=1), v]
+    blocks = [x.contiguous().view(torch.uint8).reshape(B, Hv, -1) for x in parts]
+    if cfg.gate == LQ_GATE_DIAG:
+        blocks.append(alpha.contiguous().view(torch.uint8).reshape(B, Hv, -1))
+    return torch.cat(blocks, dim=2).contiguous()
 
 
 def lq_decode_tokens(cfg, ntok: int, q, k, v, alpha, beta, state: lq_state, out, active=None,

@@ -210,6 +210,29 @@ lq_status lq_decode_step(const lq_config *cfg, const void *q, const void *k, con
   return from_cuda(lq::launch_decode(p, static_cast<cudaStream_t>(stream)));
 }
 
+lq_status lq_decode_step_packed(const lq_config *cfg, const void *qkva, const float *alpha,
+                                const float *beta, const lq_state *st, void *out,
+                                const int32_t *active, void *stream) {
+  lq_status s = check_config(cfg);
+  if (s != LQ_OK) return s;
+  if ((s = check_state(cfg, st)) != LQ_OK) return s;
+  if (cfg->window > lq::kMaxWindow) return LQ_ERR_UNSUPPORTED;
+  const bool kda = cfg->gate == LQ_GATE_DIAG;
+  if (!qkva || !beta || !out || (!kda && !alpha)) return LQ_ERR_INVALID_ARG;
+  if (!aligned16(qkva) || (!kda && !aligned_to(alpha, 4)) || !aligned_to(beta, 4) ||
+      !aligned_to(out, out_size(cfg)) || !aligned_to(active, 4))
+    return LQ_ERR_MISALIGNED;
+  if (cfg->batch == 0) return LQ_OK;
+  KParams p = make_params(cfg, st);
+  p.q = qkva;
+  p.alpha = kda ? nullptr : alpha;
+  p.beta = beta;
+  p.out = out;
+  p.mask = active;
+  p.packed = 1;
+  return from_cuda(lq::launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
 lq_status lq_decode_tokens(const lq_config *cfg, int32_t ntok, const void *q, const void *k,
                            const void *v, const float *alpha, const float *beta,
                            const lq_state *st, void *out, const int32_t *active, void *stream) {

@@ -134,7 +134,7 @@ struct SL {
     q = bg + BG;
     k = q + D * IB;
     v = k + D * IB;
-    a = v + D * IB;
+    a = v + D * IB;  // q, k, v and the gate back to back (packed inputs arrive in one copy)
     bytes = (rec_bytes + TAIL + 127) / 128 * 128;
   }
 };
@@ -980,6 +980,13 @@ __device__ __forceinline__ void issue_rest(const KParams &p, uint8_t *slot,
   }
   if (!KDA) bulk_g2s(slot + lay.bg, p.buf_g + static_cast<size_t>(tile) * kGdnGateStride,
                      bg_b, bar);
+  if (p.packed) {
+    // the slot holds q | k | v | gate back to back, as the packed inputs do
+    const uint32_t pb = 3 * in_b + (KDA ? static_cast<uint32_t>(D) * 4 : 0u);
+    bulk_g2s(slot + lay.q, static_cast<const uint8_t *>(p.q) + static_cast<size_t>(tile) * pb, pb,
+             bar);
+    return;
+  }
   const size_t qk = (static_cast<size_t>(b) * p.Hk + hk) * D * L::IB;
   bulk_g2s(slot + lay.q, static_cast<const uint8_t *>(p.q) + qk, in_b, bar);
   bulk_g2s(slot + lay.k, static_cast<const uint8_t *>(p.k) + qk, in_b, bar);

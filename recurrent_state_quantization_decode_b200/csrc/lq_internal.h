@@ -55,6 +55,7 @@ struct KParams {
   int withhold;         // decode, testing only: CTA 0 issues no copies for its first slot
   int gstride;          // floats per tile of the GDN gate buffer (gdn_gate_stride(W))
   int ntok;             // tokens per launch of the per-tile kernel (lq_decode_tokens)
+  int packed;           // decode: q holds each tile's q | k | v (| KDA gate) back to back
 };
 
 constexpr uint32_t kWaitLimitDefault = 1u << 24;

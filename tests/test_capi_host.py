@@ -27,7 +27,7 @@ def _declared():
 
 def test_exports_every_declared_symbol(B):
     names = _declared()
-    assert len(names) == 18
+    assert len(names) == 19
     assert sorted(B.EXPORTED) == names
     for n in names:
         assert hasattr(B._lib, n), n
@@ -93,6 +93,25 @@ def test_bad_pointers_rejected_before_launch(B):
         B.lq_decode_step_host(cfg, good, good, good, good, good, st, good, None, stream=0)
     assert ei.value.status == B.LQ_ERR_INVALID_ARG
     assert B.lq_get_last_error(B.lq_state(0, 0, 0, 0, 0, 0), 0) == B.LQ_ERR_INVALID_ARG
+    # packed inputs: the block pointer, GDN's separate gates and beta are required
+    # and aligned; windows above 16 tokens are refused
+    with pytest.raises(B.LQError) as ei:
+        B.lq_decode_step_packed(cfg, None, good, good, st, good, stream=0)
+    assert ei.value.status == B.LQ_ERR_INVALID_ARG
+    with pytest.raises(B.LQError) as ei:
+        B.lq_decode_step_packed(cfg, good, None, good, st, good, stream=0)
+    assert ei.value.status == B.LQ_ERR_INVALID_ARG
+    with pytest.raises(B.LQError) as ei:
+        B.lq_decode_step_packed(cfg, good + 8, good, good, st, good, stream=0)
+    assert ei.value.status == B.LQ_ERR_MISALIGNED
+    kda = B.make_config(2, 2, 2, 64, gate=B.LQ_GATE_DIAG)
+    with pytest.raises(B.LQError) as ei:                  # KDA: gates inside the blocks
+        B.lq_decode_step_packed(kda, good, None, good + 2, st, good, stream=0)
+    assert ei.value.status == B.LQ_ERR_MISALIGNED
+    w32 = B.make_config(2, 2, 4, 64, 32)
+    with pytest.raises(B.LQError) as ei:
+        B.lq_decode_step_packed(w32, good, good, good, st, good, stream=0)
+    assert ei.value.status == B.LQ_ERR_UNSUPPORTED
 
 
 def test_empty_batch_is_a_no_op(B):

@@ -311,6 +311,48 @@ def test_active_mask_and_flush(case):
     assert B.lq_get_last_error(ds.st) == B.LQ_OK
 
 
+PACKED_CASES = {
+    "kda_d128_bf16": wl.Workload("pk", 6, 32, 32, 128, wl.GATE_DIAG, True, 20),
+    "gdn_gva_d128_bf16": wl.Workload("pg", 6, 16, 32, 128, wl.GATE_SCALAR, True, 20),
+    "gdn_d64_f32": wl.Workload("pf", 5, 2, 4, 64, wl.GATE_SCALAR, False, 20),
+    "kda_d64_bf16": wl.Workload("pd", 5, 4, 4, 64, wl.GATE_DIAG, True, 20),
+}
+
+
+@pytest.mark.parametrize("case", sorted(PACKED_CASES))
+def test_packed_inputs_match_separate_inputs(case):
+    """lq_decode_step_packed on per-tile blocks and lq_decode_step on separate
+    arrays: the same bits (outputs, phases, records, buffers) over 20 tokens,
+    a fold and a random active mask included."""
+    w = PACKED_CASES[case]
+    rng = np.random.default_rng(12)
+    S0, _, _ = wl.initial_states(rng, w.tiles, w.d, w.d)
+    ti = wl.token_inputs(rng, w, w.steps)
+    active = rng.random((w.steps, w.batch)) < 0.8
+    cfg = B.config_for(w)
+    S0_dev = torch.from_numpy(S0).cuda()
+    a, b = B.DeviceState(cfg), B.DeviceState(cfg)
+    for ds in (a, b):
+        B.lq_state_init(cfg, S0_dev, ds.st)
+    dev = P.DeviceInputs(ti, w.io_bf16)
+    outs = [torch.empty((w.batch, w.num_v_heads, w.d), device="cuda") for _ in range(2)]
+    kda = w.gate == wl.GATE_DIAG
+    for t in range(w.steps):
+        act = torch.from_numpy(active[t].astype(np.int32)).cuda()
+        q, k, v, al, be = dev.token(t)
+        blocks = B.pack_tile_inputs(cfg, q, k, v, al)
+        for o in outs:
+            o.fill_(float("nan"))
+        B.lq_decode_step(cfg, q, k, v, al, be, a.st, outs[0], active=act)
+        B.lq_decode_step_packed(cfg, blocks, None if kda else al, be, b.st, outs[1], active=act)
+        assert torch.equal(outs[0].isnan(), outs[1].isnan())
+        assert torch.equal(outs[0].nan_to_num(), outs[1].nan_to_num()), t
+    for name in ("records", "buf_k", "buf_d", "buf_g", "buf_n"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    for ds in (a, b):
+        assert B.lq_get_last_error(ds.st) == B.LQ_OK
+
+
 @pytest.mark.parametrize("window,T", [(16, 21), (32, 45)])
 def test_dequantize_base_and_current_state(window, T):
     w = wl.Workload("q", 2, 2, 2, 64, wl.GATE_DIAG, False, T, window=window)
