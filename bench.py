@@ -396,15 +396,12 @@ class Layer:
         self.alpha = torch.from_numpy(ti.alpha).to(device)
         self.beta = torch.from_numpy(ti.beta).to(device)
         self.out = torch.empty((w.batch, w.num_v_heads, w.d), dtype=torch.float32, device=device)
-        # Without grouped heads (Hv = Hk) each token's inputs are also kept in
-        # lq_decode_step_packed's per-tile blocks, which the int8 step reads
-        # (one copy per tile instead of four); with grouped heads the blocks
-        # would repeat q and k per value head, so those layers keep the
-        # separate arrays.
-        self.packed = None
-        if w.num_v_heads == w.num_k_heads:
-            self.packed = [B.pack_tile_inputs(self.cfg, self.q[t], self.k[t], self.v[t],
-                                              self.alpha[t]) for t in range(w.window)]
+        # Each token's inputs are also kept in lq_decode_step_packed's per-tile
+        # blocks, which the int8 step reads: one copy per tile instead of three
+        # or four.  With grouped heads (Hv > Hk) the blocks repeat q and k per
+        # value head, more bytes than the shared arrays, and still faster.
+        self.packed = [B.pack_tile_inputs(self.cfg, self.q[t], self.k[t], self.v[t],
+                                          self.alpha[t]) for t in range(w.window)]
         self.host = None
         if phases is not None:
             ph = torch.as_tensor(phases, dtype=torch.int32, device=device)
@@ -569,7 +566,7 @@ def measure_decode(B, w: wl.Workload, key: str, L: int, steps: int, warmup: int,
     def step_int8(s):
         for t in range(W):
             for ly in layers:
-                if ly.packed is not None:
+                if ly.packed is not None:  # (always; None leaves the separate arrays)
                     kda = ly.cfg.gate == B.LQ_GATE_DIAG
                     B.lq_decode_step_packed(ly.cfg, ly.packed[t], None if kda else ly.alpha[t],
                                             ly.beta[t], ly.ds.st, ly.out, stream=s)
